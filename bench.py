@@ -1,0 +1,500 @@
+"""Benchmark of the DSA hot path (lightning indexer -> top-K -> sparse MLA) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl dsa|reference]
+
+One step is one pass of the whole hot path over one batch of synthetic, seeded input: indexer
+scores (dsa_indexer_scores), top-K selection (dsa_topk_select) and sparse MLA
+(dsa_sparse_mla_decode, or dsa_sparse_mla_prefill for the prefill chunk).  The default workload
+is bf16 decode at batch 1, context 32768 (indexer 64 heads x 128, top-2048, MLA 128 heads over
+512 + 64).  Other workloads: tiny, batched_decode, prefill, long_decode (see dsa_inputs.py).
+
+Timing: W untimed warm-up steps; then K steps, each bracketed by CUDA events on the launching
+stream, with the L2 flushed (a 256 MiB write) before every step when the workload's resident
+data fits in L2; barrier + synchronize on both sides; the max over ranks.  Rank 0 prints one
+JSON line.  With --gpus N > 1 (torchrun) every rank runs an independent replica of the workload
+(the path shards by request with no exchange step): value = all ranks' query tokens / max time.
+
+--impl reference times the fp64 CPU oracle (the method's plain definition) on this host's cores
+on a bounded sample of the same workload and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "DSA layer µs and query-tokens/s; achieved HBM TB/s / tensor util vs B200 peak"
+L2_BYTES = 126 * 1024 * 1024
+FLUSH_BYTES = 256 * 1024 * 1024
+
+# ---------------------------------------------------------------------------------------------
+# analytic model: algorithmic bytes and FLOPs of each step (method's own work, no re-reads)
+# ---------------------------------------------------------------------------------------------
+
+
+def mla_decode_arithmetic_intensity(H, d, r, b):
+    """FLOP per byte of MQA-mode MLA decode for L >> H (page "How GLM5.3 Sparse Attention Affects
+    HBM Memory Usage", section "MLA Modifications"): 2 H (2d + r) / (b (d + r))."""
+    return 2.0 * H * (2 * d + r) / (b * (d + r))
+
+
+def ridge(tflops, tbs):
+    """Ridge point in FLOP/B of a machine with the given TFLOP/s and TB/s."""
+    return tflops / tbs
+
+
+def key_bytes_per_token(spec):
+    return {"f32": 4, "bf16": 2, "e4m3": 1}[spec.key_dtype] * spec.Di + (4 if spec.key_dtype == "e4m3" else 0)
+
+
+def work_model(spec):
+    """Per-step algorithmic work of each kernel.  Units: bytes and FLOPs."""
+    act = 4 if spec.act_dtype == "f32" else 2
+    T = spec.T
+    vis = [p + 1 for p in spec.q_pos]
+    pairs = sum(vis)                                    # visible (query, key) pairs
+    # keys each request must stream once (decode: one query per request)
+    per_req = {}
+    for t in range(T):
+        r = spec.q_req[t]
+        per_req[r] = max(per_req.get(r, 0), vis[t])
+    key_tokens = sum(per_req.values())
+    idx_bytes = key_tokens * key_bytes_per_token(spec) + T * spec.Hi * (spec.Di * act + 4) + pairs * 4
+    idx_flops = 2.0 * pairs * spec.Hi * spec.Di
+    sel = [min(v, spec.k) for v in vis]
+    topk_bytes = pairs * 4 + T * spec.k * 4
+    mla_rows = sum(sel)
+    mla_bytes = mla_rows * spec.dqk * act + T * spec.H * (spec.dqk + spec.d_v) * act + T * spec.H * 4
+    mla_flops = 2.0 * spec.H * mla_rows * (spec.dqk + spec.d_v)
+    return dict(indexer_bytes=idx_bytes, indexer_flops=idx_flops, topk_bytes=topk_bytes,
+                mla_bytes=mla_bytes, mla_flops=mla_flops, key_tokens=key_tokens, pairs=pairs,
+                mla_rows=mla_rows)
+
+
+def resident_bytes(spec, x):
+    tot = 0
+    for k in ("key_pool", "key_scale", "latent_pool", "q_idx", "q_mla", "w"):
+        v = x.get(k)
+        if v is not None:
+            tot += v.numel() * v.element_size()
+    return tot
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def ncu_traffic(kernel, workload):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None when there is
+    none for this kernel and workload, or when the kernel's source changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d.get("%s@%s" % (kernel, workload))
+        if not e:
+            return None
+        src = os.path.join(ROOT, e["source"])
+        import hashlib
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if h != e["source_sha"]:
+            return None
+        return float(e["bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------------
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# CUDA arm
+# ---------------------------------------------------------------------------------------------
+
+
+def _dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def max_over_ranks(value, world, device=None):
+    """Max of a per-rank float over all ranks (identity for a single process)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(units_per_rank, max_time_s, world):
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    return units_per_rank * world / max_time_s
+
+
+class Layer:
+    """Buffers and calls of one hot-path step for a generated workload (all on the device)."""
+
+    def __init__(self, x):
+        import torch
+        import sparse_attention_06_b200 as dsa
+        self.dsa = dsa
+        self.x = x
+        spec = x["spec"]
+        self.spec = spec
+        self.keys = dsa.PagedCache(x["key_pool"], x.get("key_scale"))
+        self.lat = dsa.PagedCache(x["latent_pool"])
+        self.max_ctx = max(spec.q_pos) + 1
+        self.batch = dsa.Batch(x["q_req"], x["q_pos"], x["block_table"], self.max_ctx, spec.query_group)
+        self.ld = (self.max_ctx + 3) // 4 * 4
+        dev = x["key_pool"].device
+        self.scores = torch.empty((spec.T, self.ld), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((spec.T, spec.k), dtype=torch.int32, device=dev)
+        self.out = torch.empty((spec.T, spec.H, spec.d_v), dtype=x["q_mla"].dtype, device=dev)
+        self.lse = torch.empty((spec.T, spec.H), dtype=torch.float32, device=dev)
+        ws = dsa.dsa_mla_workspace_size(spec.T, spec.H, spec.d_v, spec.k)
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=dev) if ws else None
+        self.prefill = spec.query_group > 1
+        self.q_idx, self.w, self.q_mla = x["q_idx"], x["w"], x["q_mla"]
+
+    def step(self, ev=None):
+        d = self.dsa
+        d.dsa_indexer_scores(self.q_idx, self.w, self.keys, self.batch, self.scores)
+        if ev is not None:
+            ev[0].record()
+        d.dsa_topk_select(self.scores, self.batch.q_pos, self.spec.k, self.idx)
+        if ev is not None:
+            ev[1].record()
+        fn = d.dsa_sparse_mla_prefill if self.prefill else d.dsa_sparse_mla_decode
+        fn(self.q_mla, self.lat, self.batch, self.idx, self.spec.scale, self.out, self.lse, self.ws)
+
+
+def run_cuda(args):
+    import torch
+    rank, local_rank, world = _dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import dsa_inputs as di
+    import sparse_attention_06_b200 as dsa
+    dsa.load_library()
+    spec = di.WORKLOADS[args.config]()
+    x = di.generate(spec, device=dev)
+    layer = Layer(x)
+    model = work_model(spec)
+    flush = resident_bytes(spec, x) < 2 * L2_BYTES
+    flush_buf = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev) if flush else None
+    stream = torch.cuda.current_stream()
+
+    dsa.dsa_clear_device_error()
+    for _ in range(args.warmup):
+        layer.step()
+    torch.cuda.synchronize()
+    err = dsa.dsa_get_device_error()
+    if err:
+        raise RuntimeError("device error word %d after warm-up" % err)
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    sampler = ClockSampler(local_rank) if rank == 0 or True else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    launches0 = dsa.dsa_kernel_launch_count()
+    sampler.start()
+    for i in range(K):
+        if flush:
+            flush_buf.fill_(i)
+        e = evs[i]
+        e[0].record(stream)
+        layer.step(ev=(e[1], e[2]))
+        e[3].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    launches = dsa.dsa_kernel_launch_count() - launches0
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    idx_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    topk_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    mla_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_s = max_over_ranks(sum(step_ms) / 1e3, world, dev)
+    units = spec.T * K
+    value = aggregate(units, total_s, world)
+    ms_per_step = total_s * 1e3 / K
+
+    # end to end through the public API: per-step query-side inputs from pinned host memory,
+    # the KV caches resident in HBM (state), output read back every step
+    host_in = {n: x[n].cpu().pin_memory() for n in ("q_idx", "w", "q_mla", "q_req", "q_pos", "block_table")}
+    host_out = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+    dev_in = {n: x[n] for n in host_in}
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        if flush:
+            flush_buf.fill_(i)
+        e2e_ev[i][0].record(stream)
+        for n, t in host_in.items():
+            dev_in[n].copy_(t, non_blocking=True)
+        layer.step()
+        host_out.copy_(layer.out, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_s = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / 1e3, world, dev)
+    e2e_value = aggregate(units, e2e_s, world)
+    err = dsa.dsa_get_device_error()
+
+    # roofline of the dominant kernel (the indexer: HBM-bound in decode, tensor-bound in prefill)
+    peaks = load_peaks()
+    idx_avg_s = statistics.mean(idx_ms) / 1e3
+    if spec.query_group > 1:
+        achieved = model["indexer_flops"] / idx_avg_s / 1e12
+        peak = peaks["bf16_tflops_sustained"] if statistics.mean(step_ms) > 50 else peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak}
+    else:
+        achieved = model["indexer_bytes"] / idx_avg_s / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
+    roof["kernel"] = "indexer"
+    roof["peak_source"] = peaks["source"]
+    roof["traffic"] = ncu_traffic("indexer", args.config)
+    breakdown = {
+        "indexer_us": statistics.mean(idx_ms) * 1e3,
+        "topk_us": statistics.mean(topk_ms) * 1e3,
+        "mla_us": statistics.mean(mla_ms) * 1e3,
+        "indexer_GBps": model["indexer_bytes"] / idx_avg_s / 1e9,
+        "mla_GBps": model["mla_bytes"] / (statistics.mean(mla_ms) / 1e3) / 1e9,
+        "mla_TFLOPps": model["mla_flops"] / (statistics.mean(mla_ms) / 1e3) / 1e12,
+        "layer_us": ms_per_step * 1e3,
+    }
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(x, spec, budget_s=args.cpu_budget)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "query-tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if spec.act_dtype == "bf16" else "f32",
+            "data": "synthetic (seeded N(0,1) queries/keys/latent, U(0,1) head weights, shuffled 64-token pages)",
+            "config": {"workload": spec.name, "queries_per_step": spec.T, "requests": spec.B,
+                       "context": max(spec.lens), "indexer": "%dx%d %s keys" % (spec.Hi, spec.Di, spec.key_dtype),
+                       "top_k": spec.k, "mla": "%d heads, %d+%d" % (spec.H, spec.d_v, spec.d_rope),
+                       "l2": "flushed (256 MiB write) before every step" if flush else "inputs larger than L2",
+                       "parallelism": "replicas x%d" % world},
+            "e2e": {"value": e2e_value, "unit": "query-tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h,
+                    "note": "query-side inputs copied from pinned host memory every step; KV caches resident"},
+            "gpu_launches": launches,
+            "roofline": roof,
+            "breakdown": breakdown,
+            "cpu_baseline": cpu,
+            "clocks": clocks,
+            "device_error": err,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle: the cpu_baseline leg and the --impl reference arm
+# ---------------------------------------------------------------------------------------------
+
+
+def oracle_step(sub, spec, nthreads):
+    """One pass of the oracle over the queries in `sub` (indexer, selection, sparse MLA)."""
+    import oracle
+    s = oracle.indexer_scores(sub["q_idx"], sub["w"], sub["key_pool"], sub["key_scale"], sub["block_table"],
+                              sub["q_req"], sub["q_pos"], nthreads=nthreads)
+    idx = oracle.topk(s, sub["q_pos"], spec.k, nthreads=nthreads)
+    oracle.sparse_mla(sub["q_mla"], sub["latent_pool"], sub["block_table"], sub["q_req"], idx, spec.d_v,
+                      spec.scale, nthreads=nthreads)
+
+
+def _sample_queries(spec, budget_pairs):
+    """Queries of a bounded sample: evenly spaced over the batch, up to `budget_pairs` visible
+    (query, key) pairs."""
+    T = spec.T
+    order = [int(round(i * (T - 1) / max(1, T - 1))) for i in range(T)]
+    if T > 1:
+        stride = max(1, T // 64)
+        order = list(range(0, T, stride))
+    qs, pairs = [], 0
+    for t in order:
+        qs.append(t)
+        pairs += spec.q_pos[t] + 1
+        if pairs >= budget_pairs:
+            break
+    return qs
+
+
+def cpu_baseline(x, spec, budget_s=15.0, repeats=None):
+    """Time the oracle (as it stands) on the host cores on a bounded sample of the workload."""
+    import dsa_inputs as di
+    import oracle
+    cores = oracle.max_threads()
+    # about 1e8 fp64 MAC/s per core in the indexer loop: size the sample to the budget
+    budget_pairs = max(1, int(budget_s * cores * 1e8 / (spec.Hi * spec.Di + 1)))
+    qs = _sample_queries(spec, budget_pairs)
+    sub = di.subset(x, qs)
+    threads = min(cores, len(qs))
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle_step(sub, spec, threads)
+        n += 1
+        if repeats is not None and n >= repeats:
+            break
+        if repeats is None and (time.perf_counter() - t0 > budget_s / 3 or n >= 3):
+            break
+    dt = (time.perf_counter() - t0) / n
+    return {"value": len(qs) / dt, "unit": "query-tokens/s", "cores": threads, "kind": "oracle",
+            "sample": "%d of %d queries (%d visible key positions), %d pass(es), fp64" % (
+                len(qs), spec.T, sum(spec.q_pos[t] + 1 for t in qs), n)}
+
+
+def run_reference(args):
+    rank, _, world = _dist_env()
+    if rank != 0:
+        return
+    import torch
+    import dsa_inputs as di
+    spec = di.WORKLOADS[args.config]()
+    big = spec.name not in ("tiny_f32_L256",)
+    x = di.generate(spec, device="cpu") if not big or sum(spec.lens) <= 70000 else None
+    if x is None:
+        # draw the full workload only for the sampled queries' requests, on the CPU
+        x = di.generate(spec, device="cpu")
+    budget = min(args.cpu_budget, 120.0 / max(1, args.steps + args.warmup))
+    import oracle
+    cores = oracle.max_threads()
+    budget_pairs = max(1, int(budget * cores * 1e8 / (spec.Hi * spec.Di + 1)))
+    qs = _sample_queries(spec, budget_pairs)
+    sub = di.subset(x, qs)
+    threads = min(cores, len(qs))
+    for _ in range(args.warmup):
+        oracle_step(sub, spec, threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(sub, spec, threads)
+    total = time.perf_counter() - t0
+    value = len(qs) * args.steps / total
+    sample = "%d of %d queries per step (%d visible key positions), fp64" % (
+        len(qs), spec.T, sum(spec.q_pos[t] + 1 for t in qs))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "query-tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": {"workload": spec.name, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "query-tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "query-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="decode",
+                    choices=["tiny", "decode", "batched_decode", "prefill", "long_decode"])
+    ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,199 @@
+/*
+ * dsa.h -- C ABI of the DeepSeek Sparse Attention (DSA) hot path on one NVIDIA B200 (sm_100a).
+ *
+ * The method (pages "How GLM5.3 Sparse Attention Affects HBM Memory Usage" and its Chinese
+ * original on InferenceX, sections "Lightning Indexer", "Sparse MLA", "MLA Modifications"):
+ *   1. a lightning indexer scores every visible KV position s for each query token t,
+ *        I[t,s] = sum_h w[t,h] * ReLU(q[t,h,:] . k[s,:])       (multi-head query, one-head key);
+ *   2. the K highest-scoring positions are selected per query (shared by all attention heads);
+ *      a query that sees fewer than K positions keeps all of them (dense attention);
+ *   3. MLA runs in MQA ("absorbed") mode over only the selected rows of the latent KV cache:
+ *      each row is a 512-d latent plus a 64-d RoPE key; the full row is the key, its first
+ *      d_v dims are the value; all heads share the rows.
+ *
+ * Conventions shared by every entry point
+ *   - Ownership: the caller owns and allocates every buffer (device memory unless stated).
+ *     The library never allocates device memory; scratch is passed in by the caller.
+ *   - Asynchrony: every compute call only enqueues kernels on `stream` (a cudaStream_t, NULL for
+ *     the legacy default stream) and returns; there is no host synchronisation inside a call,
+ *     except in dsa_get_device_error, which is documented as synchronous.
+ *   - Positions: query t belongs to request q_req[t] and sits at absolute position q_pos[t];
+ *     it sees positions 0..q_pos[t] of its request (causal, including itself).  Selected
+ *     indices are logical positions within the request; only kernels that read a paged cache
+ *     apply the block table: row = block_table[req][pos / block_size] * block_size
+ *     + pos % block_size.
+ *   - Errors: shapes, dtypes, alignment and NULL pointers are checked on the host before
+ *     anything is launched (DSA_ERR_INVALID_ARG); valid but unimplemented combinations return
+ *     DSA_ERR_UNSUPPORTED; a failed launch returns DSA_ERR_CUDA.  Faults that only the device
+ *     can see (a block id outside the pool, a selected index outside 0..q_pos, a request id
+ *     outside the batch, a NaN score, a bounded wait that ran out) never trap: the kernel sets
+ *     a bit in the library's device error word (DSA_DEVERR_*), skips the offending element,
+ *     and the host reads the word with dsa_get_device_error.
+ *   - Tensor cores: production shapes (indexer 64 heads x 128, MLA 128 heads over 512 + 64,
+ *     bf16 operands, e4m3 or bf16 indexer keys) run on tcgen05/TMA kernels; any other shape runs
+ *     on a generic CUDA-core path of the same library.  There is no CPU fallback.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA_ABI_VERSION 1
+
+typedef enum dsa_status {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,
+  DSA_ERR_UNSUPPORTED = 2,
+  DSA_ERR_CUDA = 3,
+  DSA_ERR_DEVICE_FAULT = 4
+} dsa_status;
+
+typedef enum dsa_dtype {
+  DSA_F32 = 0,
+  DSA_BF16 = 1,
+  DSA_E4M3 = 2 /* OCP FP8 E4M3 ("fn": no infinities), used with a per-token f32 scale */
+} dsa_dtype;
+
+/* Bits of the device error word. */
+#define DSA_DEVERR_BLOCK_ID 1      /* block_table entry outside [0, num_blocks) */
+#define DSA_DEVERR_INDEX 2         /* selected index outside [-1, q_pos[t]] */
+#define DSA_DEVERR_REQUEST 4       /* q_req[t] outside [0, num_reqs) or q_pos[t] >= max_context */
+#define DSA_DEVERR_NAN_SCORE 8     /* NaN indexer score met by the selection */
+#define DSA_DEVERR_TIMEOUT 16      /* a bounded wait inside a kernel gave up */
+#define DSA_DEVERR_QUERY_GROUP 32  /* queries of one group are not in one request */
+
+typedef void* dsa_stream; /* cudaStream_t */
+
+/* A paged per-token cache: `data` is [num_blocks, block_size, dim] of `dtype`, row-major, in
+ * device memory, 16-byte aligned, one token per row.  For DSA_E4M3, `scale` is the per-token
+ * dequantisation scale [num_blocks, block_size] f32 (value = code * scale, scale > 0); it is
+ * NULL for the other dtypes.  block_size is 64. */
+typedef struct dsa_paged_cache {
+  const void* data;
+  const float* scale;
+  int64_t num_blocks;
+  int32_t block_size;
+  int32_t dim;
+  int32_t dtype; /* dsa_dtype */
+  int32_t reserved;
+} dsa_paged_cache;
+
+/* The queries of one call.  q_req, q_pos and block_table are device int32 arrays:
+ * q_req [num_queries], q_pos [num_queries], block_table [num_reqs, max_blocks].
+ * max_context is a host-side bound: every q_pos[t] < max_context (it sizes score rows).
+ * query_group G >= 1 is a host-side promise that queries come in runs of G consecutive t
+ * (num_queries a multiple of G) sharing one request; a prefill chunk passes 4, decode passes 1.
+ * It only selects kernels: a broken promise sets DSA_DEVERR_QUERY_GROUP. */
+typedef struct dsa_batch {
+  int32_t num_queries;
+  int32_t num_reqs;
+  const int32_t* q_req;
+  const int32_t* q_pos;
+  const int32_t* block_table;
+  int32_t max_blocks;
+  int32_t max_context;
+  int32_t query_group;
+  int32_t reserved;
+} dsa_batch;
+
+/*
+ * Lightning-indexer scores (page "How GLM5.3 Sparse Attention Affects HBM Memory Usage",
+ * section "Lightning Indexer": dot product, ReLU, weighted sum over the query heads; no value,
+ * no softmax).
+ *   scores[t * ld + s] = sum_h w[t,h] * max(0, sum_i q[t,h,i] * khat[s,i]),  0 <= s <= q_pos[t]
+ *   khat = key row (f32/bf16), or e4m3 code * per-token scale.
+ * q: device [num_queries, Hi, Di] of q_dtype (DSA_F32 or DSA_BF16); w: device [num_queries, Hi]
+ * f32; keys: paged indexer-key cache with dim == Di, same block table as the batch;
+ * scores: device f32 [num_queries, ld], ld >= max_context.  Entries s > q_pos[t] are not
+ * written.  Fast path: Hi == 64, Di == 128, bf16 q, bf16 or e4m3 keys.
+ */
+dsa_status dsa_indexer_scores(const void* q, int32_t q_dtype, int32_t Hi, int32_t Di,
+                              const float* w, const dsa_paged_cache* keys,
+                              const dsa_batch* batch, float* scores, int64_t ld,
+                              dsa_stream stream);
+
+/*
+ * Top-K selection (same page, section "Lightning Indexer": the K highest indexer scores are
+ * kept per query and shared by all heads; a query seeing fewer than K positions keeps all).
+ * For query t with n = q_pos[t] + 1 visible scores scores[t * ld + 0 .. n-1]:
+ *   n <= k: idx[t] = 0, 1, ..., n-1, then -1;
+ *   n >  k: the k positions first in the order (score descending, position ascending), written
+ *           in ascending position order.
+ * -0.0 and +0.0 are equal scores; a NaN score sets DSA_DEVERR_NAN_SCORE (it ranks lowest).
+ * scores: device f32 [T, ld]; q_pos: device int32 [T] with q_pos[t] < ld (a larger value sets
+ * DSA_DEVERR_REQUEST and only the first ld scores are used); idx: device int32 [T, k].
+ * k in [1, 4096].  Needs no scratch memory.
+ */
+dsa_status dsa_topk_select(const float* scores, int64_t ld, const int32_t* q_pos, int32_t T,
+                           int32_t k, int32_t* idx, dsa_stream stream);
+
+/*
+ * Indexer scores followed by the top-K selection, in one call.  `scores` is caller-owned
+ * scratch of [num_queries, ld] f32 (ld >= max_context) that receives the scores; idx is
+ * device int32 [num_queries, k].  Same arguments and semantics as the two calls above.
+ */
+dsa_status dsa_indexer_topk(const void* q, int32_t q_dtype, int32_t Hi, int32_t Di,
+                            const float* w, const dsa_paged_cache* keys,
+                            const dsa_batch* batch, int32_t k, float* scores, int64_t ld,
+                            int32_t* idx, dsa_stream stream);
+
+/*
+ * Sparse MLA in MQA mode over the selected rows (same page, sections "Sparse MLA" and "MLA
+ * Modifications": P = Q[H, d+r] K^T over the selected latent rows, O = P V, where V is the
+ * first d of each row; the softmax is the usual scaled one).  For query t and head h:
+ *   logit_j = softmax_scale * (q[t,h,:] . row(idx[t,j]))           (all d_v + d_rope dims)
+ *   out[t,h,:] = sum_j softmax_j(logit) * row(idx[t,j])[0:d_v]
+ *   lse[t,h]   = ln sum_j exp(logit_j)          (-inf and out = 0 when nothing is selected)
+ * Entries idx[t,j] == -1 are skipped; any other index outside 0..q_pos[t] sets
+ * DSA_DEVERR_INDEX and is skipped.
+ * q: device [num_queries, H, d_v + d_rope] of q_dtype; latent: paged cache with
+ * dim == d_v + d_rope and dtype == q_dtype (f32 or bf16); idx: device int32 [num_queries, k];
+ * out: device [num_queries, H, d_v] of q_dtype; lse: device f32 [num_queries, H] or NULL.
+ * workspace: device scratch of at least dsa_mla_workspace_size(num_queries, H, d_v, k) bytes,
+ * 256-byte aligned (may be NULL when that size is 0).
+ * The decode entry point splits each query's k rows across CTAs and merges the partial
+ * results (log-sum-exp combine); the prefill entry point gives each query whole CTAs.
+ * Fast path: H == 128, d_v == 512, d_rope == 64, bf16.
+ */
+dsa_status dsa_sparse_mla_decode(const void* q, int32_t q_dtype, int32_t H, int32_t d_v,
+                                 int32_t d_rope, const dsa_paged_cache* latent,
+                                 const dsa_batch* batch, const int32_t* idx, int32_t k,
+                                 float softmax_scale, void* out, float* lse, void* workspace,
+                                 size_t workspace_bytes, dsa_stream stream);
+
+dsa_status dsa_sparse_mla_prefill(const void* q, int32_t q_dtype, int32_t H, int32_t d_v,
+                                  int32_t d_rope, const dsa_paged_cache* latent,
+                                  const dsa_batch* batch, const int32_t* idx, int32_t k,
+                                  float softmax_scale, void* out, float* lse, void* workspace,
+                                  size_t workspace_bytes, dsa_stream stream);
+
+/* Bytes of workspace dsa_sparse_mla_decode needs for these sizes (0 when none). Host only. */
+size_t dsa_mla_workspace_size(int32_t num_queries, int32_t H, int32_t d_v, int32_t k);
+
+/* Synchronises `stream`, then reads the device error word of the current device into *code
+ * (0 = no fault).  Not for use inside stream capture. */
+dsa_status dsa_get_device_error(int32_t* code, dsa_stream stream);
+
+/* Enqueues a reset of the current device's error word to 0 on `stream`. */
+dsa_status dsa_clear_device_error(dsa_stream stream);
+
+/* Static description of a status code; detail of the last failed call on this host thread. */
+const char* dsa_status_string(dsa_status status);
+const char* dsa_last_error_message(void);
+
+int32_t dsa_abi_version(void);
+
+/* Number of kernels this library has enqueued in this process so far (all devices).  Host only;
+ * a diagnostic for counting launches inside a timed region. */
+int64_t dsa_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

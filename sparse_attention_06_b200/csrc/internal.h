@@ -1,0 +1,61 @@
+// internal.h -- launchers shared between the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/dsa.h"
+
+namespace dsa {
+
+// Arguments of an indexer launch after host validation.
+struct IndexerArgs {
+  const void* q;
+  int q_dtype;
+  int Hi, Di;
+  const float* w;
+  dsa_paged_cache keys;
+  dsa_batch batch;
+  float* scores;
+  int64_t ld;
+  int* err;
+};
+
+struct MlaArgs {
+  const void* q;
+  int dtype;
+  int H, d_v, d_rope;
+  dsa_paged_cache latent;
+  dsa_batch batch;
+  const int32_t* idx;
+  int k;
+  float scale;
+  void* out;
+  float* lse;
+  void* workspace;
+  size_t workspace_bytes;
+  int* err;
+};
+
+// generic CUDA-core path (any shape)
+cudaError_t launch_indexer_generic(const IndexerArgs& a, cudaStream_t s);
+cudaError_t launch_mla_generic(const MlaArgs& a, cudaStream_t s);
+
+// radix top-k (any k <= 4096)
+cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, int T, int k,
+                        int32_t* idx, int* err, cudaStream_t s);
+
+// tcgen05 paths (production shapes)
+cudaError_t launch_indexer_tc_decode(const IndexerArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_indexer_tc_prefill(const IndexerArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_t s);
+int mla_tc_num_splits(int T, int k, int num_sms);
+size_t mla_tc_workspace_bytes(int T, int H, int d_v, int nsplit);
+
+// tensor-map encoding through the driver entry point (no link-time libcuda dependency)
+bool encode_tmap_2d(void* tmap_out, const void* base, int elem_bytes, uint64_t inner,
+                    uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
+                    uint32_t box_outer, bool swizzle128);
+
+}  // namespace dsa

@@ -1,0 +1,86 @@
+"""The C ABI library builds, loads and exports every entry point include/dsa.h declares; host-side
+argument checks reject bad calls before anything touches CUDA.  No compute calls (no GPU here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_attention_06_b200 as dsa
+from sparse_attention_06_b200 import build as dsa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dsa_build.build()
+    return dsa.load_library()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert "dsa_indexer_scores" in names and "dsa_sparse_mla_prefill" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(dsa.EXPORTED) <= set(names)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.dsa_abi_version() == 1
+    assert lib.dsa_status_string(dsa.DSA_ERR_INVALID_ARG) == b"invalid argument"
+
+
+def test_invalid_arguments_rejected_on_host(lib):
+    # NULL batch
+    st = lib.dsa_indexer_scores(None, 1, 64, 128, None, None, None, None, 0, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+    assert b"batch" in lib.dsa_last_error_message()
+    # k out of range / NULL pointers in the selection
+    assert lib.dsa_topk_select(None, 10, None, 1, 5, None, None) == dsa.DSA_ERR_INVALID_ARG
+    fake = ctypes.c_void_p(16)
+    assert lib.dsa_topk_select(fake, 10, fake, 1, 0, fake, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_topk_select(fake, 10, fake, 1, 5000, fake, None) == dsa.DSA_ERR_INVALID_ARG
+    # query_group must divide num_queries
+    b = dsa._Batch(6, 1, 16, 16, 16, 4, 256, 4, 0)
+    kc = dsa._PagedCache(16, None, 4, 64, 128, dsa.DSA_BF16, 0)
+    st = lib.dsa_indexer_scores(fake, 1, 64, 128, fake, ctypes.byref(kc), ctypes.byref(b), fake, 256, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG and b"query_group" in lib.dsa_last_error_message()
+    # e4m3 cache without a scale
+    b = dsa._Batch(1, 1, 16, 16, 16, 4, 256, 1, 0)
+    kc = dsa._PagedCache(16, None, 4, 64, 128, dsa.DSA_E4M3, 0)
+    st = lib.dsa_indexer_scores(fake, 1, 64, 128, fake, ctypes.byref(kc), ctypes.byref(b), fake, 256, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG and b"scale" in lib.dsa_last_error_message()
+    # latent dim must be d_v + d_rope; scale must be positive
+    lc = dsa._PagedCache(16, None, 4, 64, 500, dsa.DSA_BF16, 0)
+    st = lib.dsa_sparse_mla_decode(fake, 1, 128, 512, 64, ctypes.byref(lc), ctypes.byref(b), fake, 2048,
+                                   ctypes.c_float(0.07), fake, None, None, 0, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+    lc = dsa._PagedCache(16, None, 4, 64, 576, dsa.DSA_BF16, 0)
+    st = lib.dsa_sparse_mla_decode(fake, 1, 128, 512, 64, ctypes.byref(lc), ctypes.byref(b), fake, 2048,
+                                   ctypes.c_float(-1.0), fake, None, None, 0, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+    # max_blocks * block_size must cover max_context
+    b = dsa._Batch(1, 1, 16, 16, 16, 2, 256, 1, 0)
+    st = lib.dsa_sparse_mla_decode(fake, 1, 128, 512, 64, ctypes.byref(lc), ctypes.byref(b), fake, 2048,
+                                   ctypes.c_float(0.07), fake, None, None, 0, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_noop(lib):
+    b = dsa._Batch(0, 0, None, None, None, 0, 0, 1, 0)
+    assert lib.dsa_indexer_scores(None, 1, 64, 128, None, None, ctypes.byref(b), None, 0, None) == dsa.DSA_OK
+    assert lib.dsa_topk_select(None, 1, None, 0, 16, None, None) == dsa.DSA_OK
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(dsa, "LIB_PATH", str(tmp_path / "nope.so"))
+    monkeypatch.setattr(dsa, "_lib", None)
+    with pytest.raises(dsa.DsaLibraryMissing):
+        dsa.load_library()

@@ -1,0 +1,154 @@
+"""GPU parity of the CUDA path against the fp64 oracle at sizes the oracle finishes in seconds:
+several tiles, ragged tails, dense (n <= K) and sparse queries, bf16 and e4m3 keys, the tiny fp32
+layer, and the device error word.  All calls go through the C ABI."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import dsa_inputs as di
+import oracle
+import sparse_attention_06_b200 as dsa
+from _parity import TOL, check_topk, parity_case, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _spec(lens, key_dtype="bf16", k=2048, **kw):
+    return di.Spec("t", lens=lens, q_req=list(range(len(lens))), q_pos=[L - 1 for L in lens],
+                   key_dtype=key_dtype, k=k, **kw)
+
+
+def test_tiny_fp32_layer():
+    x = to_dev(di.generate(di.tiny(), "cpu"))
+    r = parity_case(x, kind="f32")
+    assert r["overlap"] == 1.0
+
+
+@pytest.mark.parametrize("key_dtype", ["bf16", "e4m3"])
+def test_decode_ragged_batch(key_dtype):
+    # request 0 is dense (n <= K), the others span several 128-key tiles with ragged tails
+    spec = _spec([300, 2049, 2100, 4133, 64], key_dtype=key_dtype, seed=11)
+    x = to_dev(di.generate(spec, "cpu"))
+    parity_case(x, kind=key_dtype)
+
+
+def test_decode_small_k_many_tiles():
+    spec = _spec([1000, 777], k=100, seed=12)
+    x = to_dev(di.generate(spec, "cpu"))
+    parity_case(x, kind="bf16")
+
+
+@pytest.mark.parametrize("entry", ["decode", "prefill"])
+def test_prefill_chunk_e4m3(entry):
+    ctx, chunk = 1990, 96  # queries straddle the dense/sparse boundary at K = 2048
+    spec = di.Spec("p", lens=[ctx + chunk], q_req=[0] * chunk, q_pos=[ctx + t for t in range(chunk)],
+                   key_dtype="e4m3", query_group=4, seed=13)
+    x = to_dev(di.generate(spec, "cpu"))
+    parity_case(x, kind="e4m3", mla_entry=entry)
+
+
+def test_prefill_chunk_bf16_two_requests():
+    # two requests, 8 queries each, in groups of 4
+    spec = di.Spec("p2", lens=[3000, 2500], q_req=[0] * 8 + [1] * 8,
+                   q_pos=[2992 + t for t in range(8)] + [2492 + t for t in range(8)],
+                   query_group=4, seed=14)
+    x = to_dev(di.generate(spec, "cpu"))
+    parity_case(x, kind="bf16", mla_entry="prefill")
+
+
+# ---------------------------------------------------------------------------------------------
+# standalone selection
+# ---------------------------------------------------------------------------------------------
+
+def _topk_gpu(scores, qpos, k):
+    s = scores.cuda()
+    qp = torch.tensor(qpos, dtype=torch.int32, device="cuda")
+    idx = torch.empty((len(qpos), k), dtype=torch.int32, device="cuda")
+    dsa.dsa_clear_device_error()
+    dsa.dsa_topk_select(s, qp, k, idx)
+    err = dsa.dsa_get_device_error()
+    return idx.cpu(), err
+
+
+def test_topk_planted_tail_long_rows():
+    lens = [202752, 131072, 4096, 2049, 2048, 100]
+    ld = 202752
+    s = di.planted_scores(len(lens), ld, lens, seed=21)
+    idx, err = _topk_gpu(s, [L - 1 for L in lens], 2048)
+    assert err == 0
+    check_topk(idx, s, [L - 1 for L in lens], 2048)
+
+
+def test_topk_ties_and_signed_zeros():
+    g = torch.Generator().manual_seed(5)
+    T, ld = 6, 5000
+    s = torch.randint(-3, 4, (T, ld), generator=g).float()     # heavy ties
+    s[1] = 0.0
+    s[1, ::2] = -0.0                                           # +0 / -0 mix, all equal
+    s[2] = 7.5                                                 # all equal
+    s[3, :] = torch.arange(ld).float() * 0                     # zeros
+    s[4] = torch.randn(ld, generator=g).round(decimals=1)
+    s[5] = -torch.arange(ld).float()                           # strictly decreasing
+    qpos = [4999, 4999, 4000, 2500, 4999, 3000]
+    for k in (1, 17, 2048, 4096):
+        idx, err = _topk_gpu(s, qpos, k)
+        assert err == 0
+        check_topk(idx, s, qpos, k)
+    idx, _ = _topk_gpu(s, qpos, 2048)
+    assert idx[2].tolist() == list(range(2048))                # lower positions win the tie
+    assert idx[5].tolist() == list(range(2048))
+
+
+def test_topk_dense_boundary_and_padding():
+    s = torch.randn(4, 3000)
+    qpos = [0, 2046, 2047, 2048]      # n = 1, 2047, 2048 (dense) and 2049 (sparse)
+    idx, err = _topk_gpu(s, qpos, 2048)
+    assert err == 0
+    assert idx[0, 0] == 0 and (idx[0, 1:] == -1).all()
+    assert idx[1, :2047].tolist() == list(range(2047)) and idx[1, 2047] == -1
+    assert idx[2].tolist() == list(range(2048))
+    check_topk(idx, s, qpos, 2048)
+
+
+def test_topk_nan_sets_error_word():
+    s = torch.randn(1, 5000)
+    s[0, 77] = float("nan")
+    idx, err = _topk_gpu(s, [4999], 2048)
+    assert err & dsa.DEVERR_NAN_SCORE
+
+
+# ---------------------------------------------------------------------------------------------
+# device-detected faults: flagged, never trapped
+# ---------------------------------------------------------------------------------------------
+
+def test_bad_block_id_and_bad_index_flagged():
+    spec = _spec([500], k=64, seed=31)
+    x = to_dev(di.generate(spec, "cpu"))
+    bt = x["block_table"].clone()
+    bt[0, 3] = x["num_blocks"] + 5          # outside the pool
+    keys = dsa.PagedCache(x["key_pool"], None)
+    batch = dsa.Batch(x["q_req"], x["q_pos"], bt, 500)
+    scores = torch.zeros((1, 500), dtype=torch.float32, device="cuda")
+    dsa.dsa_clear_device_error()
+    dsa.dsa_indexer_scores(x["q_idx"], x["w"], keys, batch, scores)
+    assert dsa.dsa_get_device_error() & dsa.DEVERR_BLOCK_ID
+    # a selected index beyond q_pos
+    batch = dsa.Batch(x["q_req"], x["q_pos"], x["block_table"], 500)
+    idx = torch.full((1, 64), -1, dtype=torch.int32, device="cuda")
+    idx[0, 0] = 10
+    idx[0, 1] = 600
+    out = torch.empty((1, spec.H, spec.d_v), dtype=torch.bfloat16, device="cuda")
+    dsa.dsa_clear_device_error()
+    ws_bytes = dsa.dsa_mla_workspace_size(1, spec.H, spec.d_v, 64)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda") if ws_bytes else None
+    dsa.dsa_sparse_mla_decode(x["q_mla"], dsa.PagedCache(x["latent_pool"]), batch, idx, spec.scale, out,
+                              None, ws)
+    assert dsa.dsa_get_device_error() & dsa.DEVERR_INDEX
+    # the valid row still gives the single-row closed form: O = V of row 10
+    flat = x["latent_pool"].view(-1, spec.dqk)
+    row = flat[int(x["block_table"][0, 0]) * 64 + 10, :spec.d_v].float()
+    assert torch.allclose(out[0].float(), row.expand(spec.H, -1), atol=1e-2)
+    dsa.dsa_clear_device_error()
+    assert dsa.dsa_get_device_error() == 0
