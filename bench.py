@@ -36,6 +36,7 @@ if ROOT not in sys.path:
 METRIC = "DSA layer µs and query-tokens/s; achieved HBM TB/s / tensor util vs B200 peak"
 L2_BYTES = 126 * 1024 * 1024
 FLUSH_BYTES = 256 * 1024 * 1024
+GATE_CYCLES = 100_000_000  # ~50 ms spin at 2 GHz before the timed launches start
 
 # ---------------------------------------------------------------------------------------------
 # analytic model: algorithmic bytes and FLOPs of each step (method's own work, no re-reads)
@@ -277,6 +278,9 @@ def run_cuda(args):
     torch.cuda.synchronize()
     launches0 = dsa.dsa_kernel_launch_count()
     sampler.start()
+    # hold the stream for a moment so that every timed launch is enqueued before the device starts:
+    # the events then measure back-to-back device execution, not host launch gaps
+    torch.cuda._sleep(GATE_CYCLES)
     for i in range(K):
         if flush:
             flush_buf.fill_(i)
@@ -312,6 +316,7 @@ def run_cuda(args):
     for i in range(K):
         if flush:
             flush_buf.fill_(i)
+        torch.cuda.synchronize()  # end to end: every step starts from an idle device and host
         e2e_ev[i][0].record(stream)
         for n, t in host_in.items():
             dev_in[n].copy_(t, non_blocking=True)

@@ -416,46 +416,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// grid (T), block 128 (one thread per head): merge the split partials.
-__global__ void mla_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
-                                   int nsplit, __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out) {
-  const int t = blockIdx.x;
-  const int h = threadIdx.x & (kH - 1);
-  const int cq = threadIdx.x >> 7;  // column quarter handled by this thread
+// grid (T, 128 heads), block 128: merge the split partials of one (query, head) row; each thread
+// owns 4 of the 512 value columns.
+__global__ void __launch_bounds__(128) mla_combine_kernel(const float* __restrict__ part_o,
+                                                          const float* __restrict__ part_lse, int nsplit,
+                                                          __nv_bfloat16* __restrict__ out,
+                                                          float* __restrict__ lse_out) {
+  const int t = blockIdx.x, h = blockIdx.y, c = threadIdx.x * 4;
+  const int64_t row0 = (int64_t)t * nsplit * kH + h;  // partial row of split 0; split sp adds sp*kH
   float mx = -INFINITY;
-  for (int sp = 0; sp < nsplit; ++sp) mx = fmaxf(mx, part_lse[((int64_t)t * nsplit + sp) * kH + h]);
+  for (int sp = 0; sp < nsplit; ++sp) mx = fmaxf(mx, part_lse[row0 + (int64_t)sp * kH]);
   float wsum = 0.0f;
+  float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   for (int sp = 0; sp < nsplit; ++sp) {
-    const float ls = part_lse[((int64_t)t * nsplit + sp) * kH + h];
-    wsum += ls == -INFINITY ? 0.0f : expf(ls - mx);
+    const int64_t prow = row0 + (int64_t)sp * kH;
+    const float ls = part_lse[prow];
+    if (ls == -INFINITY) continue;
+    const float wgt = expf(ls - mx);
+    wsum += wgt;
+    const float4 a = *reinterpret_cast<const float4*>(part_o + prow * kDv + c);
+    acc.x = fmaf(wgt, a.x, acc.x);
+    acc.y = fmaf(wgt, a.y, acc.y);
+    acc.z = fmaf(wgt, a.z, acc.z);
+    acc.w = fmaf(wgt, a.w, acc.w);
   }
   const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
-  const int c_lo = cq * (kDv / 4), c_hi = c_lo + kDv / 4;
-  for (int c0 = c_lo; c0 < c_hi; c0 += 8) {
-    float acc[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
-    for (int sp = 0; sp < nsplit; ++sp) {
-      const int64_t prow = ((int64_t)t * nsplit + sp) * kH + h;
-      const float ls = part_lse[prow];
-      if (ls == -INFINITY) continue;
-      const float wgt = expf(ls - mx) * inv;
-      const float4 a = *reinterpret_cast<const float4*>(part_o + prow * kDv + c0);
-      const float4 b = *reinterpret_cast<const float4*>(part_o + prow * kDv + c0 + 4);
-      acc[0] = fmaf(wgt, a.x, acc[0]); acc[1] = fmaf(wgt, a.y, acc[1]);
-      acc[2] = fmaf(wgt, a.z, acc[2]); acc[3] = fmaf(wgt, a.w, acc[3]);
-      acc[4] = fmaf(wgt, b.x, acc[4]); acc[5] = fmaf(wgt, b.y, acc[5]);
-      acc[6] = fmaf(wgt, b.z, acc[6]); acc[7] = fmaf(wgt, b.w, acc[7]);
-    }
-    uint32_t pk[4];
-#pragma unroll
-    for (int c = 0; c < 8; c += 2) {
-      const __nv_bfloat162 hh = __floats2bfloat162_rn(acc[c], acc[c + 1]);
-      pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
-    }
-    *reinterpret_cast<uint4*>(out + ((int64_t)t * kH + h) * kDv + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  }
-  if (lse_out && cq == 0) lse_out[(int64_t)t * kH + h] = wsum > 0.0f ? mx + logf(wsum) : -INFINITY;
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  uint2 pk;
+  pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+  pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(out + ((int64_t)t * kH + h) * kDv + c) = pk;
+  if (lse_out && threadIdx.x == 0) lse_out[(int64_t)t * kH + h] = wsum > 0.0f ? mx + logf(wsum) : -INFINITY;
 }
 
 int splits_for(int T, int k, int num_sms) {
@@ -523,7 +515,7 @@ cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_
   mla_tc_kernel<<<grid, kThreads, SMEM, s>>>(qmap, p);
   e = cudaGetLastError();
   if (e != cudaSuccess || nsplit == 1) return e;
-  mla_combine_kernel<<<T, 4 * kH, 0, s>>>(p.part_o, p.part_lse, nsplit, p.out, a.lse);
+  mla_combine_kernel<<<dim3(T, kH), 128, 0, s>>>(p.part_o, p.part_lse, nsplit, p.out, a.lse);
   return cudaGetLastError();
 }
 
