@@ -1,0 +1,36 @@
+"""The benchmark's analytic model against values the article prints ("MLA Modifications" of "How
+GLM5.3 Sparse Attention Affects HBM Memory Usage"): the MQA-mode MLA decode arithmetic intensity
+2H(2d + r)/(b(d + r)) is about 2H for the V3.2 shape, 120.8 FLOP/B for GLM-5 (H = 64), and the
+H800 ridge is 865 TFLOP/s / 3.35 TB/s = 258.2 FLOP/B, which puts H near 128."""
+import pytest
+
+import bench
+import dsa_inputs as di
+
+
+def test_printed_arithmetic_intensities():
+    assert bench.mla_decode_arithmetic_intensity(64, 512, 64, 2) == pytest.approx(120.8, abs=0.1)
+    for H in (16, 64, 128):
+        assert bench.mla_decode_arithmetic_intensity(H, 512, 64, 2) == pytest.approx(2 * H, rel=0.06)
+    r = bench.ridge(865.0, 3.35)
+    assert r == pytest.approx(258.2, abs=0.05)
+    # H at the H800 ridge: 2H(2d+r)/(b(d+r)) = 258.2  ->  H ~ 128 (the article's conclusion)
+    H = r / bench.mla_decode_arithmetic_intensity(1, 512, 64, 2)
+    assert H == pytest.approx(128, rel=0.07)
+
+
+def test_work_model_decode_counts():
+    spec = di.decode()
+    m = bench.work_model(spec)
+    assert m["key_tokens"] == 32768 and m["pairs"] == 32768 and m["mla_rows"] == 2048
+    assert m["indexer_flops"] == 2 * 32768 * 64 * 128
+    assert m["mla_flops"] == 2 * 128 * 2048 * (576 + 512)
+    # keys 256 B/token + 4 B score per key + q and w once
+    assert m["indexer_bytes"] == 32768 * (256 + 4) + 64 * (128 * 2 + 4)
+
+
+def test_work_model_prefill_pairs():
+    spec = di.prefill()
+    m = bench.work_model(spec)
+    assert m["pairs"] == sum(65537 + t for t in range(4096))
+    assert m["indexer_flops"] == pytest.approx(4.54e12, rel=0.01)
