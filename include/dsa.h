@@ -172,6 +172,24 @@ dsa_status dsa_sparse_mla_prefill(const void* q, int32_t q_dtype, int32_t H, int
                                   float softmax_scale, void* out, float* lse, void* workspace,
                                   size_t workspace_bytes, dsa_stream stream);
 
+/*
+ * Sparse MLA decode without caller-provided workspace.  The pages have no counterpart: this is a
+ * convenience entry point for callers that cannot allocate device memory (for example code that
+ * runs inside another framework's memory pool, or on a path where allocation is not allowed).
+ * Same inputs, outputs and results as dsa_sparse_mla_decode; the split partials go to a fixed
+ * 32 MiB scratch array inside the library (held on every GPU that loads the library until the
+ * process exits).  Sizes whose partials need more than that return DSA_ERR_INVALID_ARG with a
+ * message (use dsa_sparse_mla_decode with a workspace then).  Allocates nothing.
+ * The first call on each device looks up the scratch address (cudaGetSymbolAddress); make that
+ * first call before any stream capture.  All calls share the scratch: calls whose kernels overlap
+ * on the GPU race; calls ordered on one stream are safe.  Nothing in the scratch needs clearing.
+ */
+dsa_status dsa_sparse_mla_decode_noalloc(const void* q, int32_t q_dtype, int32_t H, int32_t d_v,
+                                         int32_t d_rope, const dsa_paged_cache* latent,
+                                         const dsa_batch* batch, const int32_t* idx, int32_t k,
+                                         float softmax_scale, void* out, float* lse,
+                                         dsa_stream stream);
+
 /* Bytes of workspace dsa_sparse_mla_decode needs for these sizes (0 when none). Host only. */
 size_t dsa_mla_workspace_size(int32_t num_queries, int32_t H, int32_t d_v, int32_t k);
 

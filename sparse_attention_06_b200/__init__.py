@@ -34,7 +34,7 @@ EXPORTED = (
     "dsa_indexer_scores", "dsa_topk_select", "dsa_indexer_topk", "dsa_sparse_mla_decode",
     "dsa_sparse_mla_prefill", "dsa_mla_workspace_size", "dsa_get_device_error",
     "dsa_clear_device_error", "dsa_status_string", "dsa_last_error_message", "dsa_abi_version",
-    "dsa_kernel_launch_count",
+    "dsa_kernel_launch_count", "dsa_sparse_mla_decode_noalloc",
 )
 
 
@@ -82,6 +82,7 @@ def load_library():
         "dsa_indexer_topk": [P, I32, I32, I32, P, PC, PB, I32, P, I64, P, P],
         "dsa_sparse_mla_decode": [P, I32, I32, I32, I32, PC, PB, P, I32, F, P, P, P, ctypes.c_size_t, P],
         "dsa_sparse_mla_prefill": [P, I32, I32, I32, I32, PC, PB, P, I32, F, P, P, P, ctypes.c_size_t, P],
+        "dsa_sparse_mla_decode_noalloc": [P, I32, I32, I32, I32, PC, PB, P, I32, F, P, P, P],
         "dsa_get_device_error": [ctypes.POINTER(I32), P],
         "dsa_clear_device_error": [P],
     }
@@ -217,6 +218,21 @@ def dsa_sparse_mla_decode(q, latent: PagedCache, batch: Batch, idx, softmax_scal
 def dsa_sparse_mla_prefill(q, latent: PagedCache, batch: Batch, idx, softmax_scale, out, lse=None,
                            workspace=None, stream=None):
     return _mla("dsa_sparse_mla_prefill", q, latent, batch, idx, softmax_scale, out, lse, workspace, stream)
+
+
+def dsa_sparse_mla_decode_noalloc(q, latent: PagedCache, batch: Batch, idx, softmax_scale, out, lse=None,
+                                  stream=None):
+    """dsa_sparse_mla_decode for callers that cannot allocate device memory: the split partials
+    live in the library's fixed 32 MiB device scratch (see include/dsa.h)."""
+    lib = load_library()
+    T, H, dqk = q.shape
+    d_v = out.shape[-1]
+    lc, bc = latent._c(), batch._c()
+    _check(lib.dsa_sparse_mla_decode_noalloc(_dev_ptr(q, "q"), _dtype_code(q), H, d_v, dqk - d_v,
+                                             ctypes.byref(lc), ctypes.byref(bc), _dev_ptr(idx, "idx"),
+                                             idx.shape[1], float(softmax_scale), _dev_ptr(out, "out"),
+                                             _dev_ptr(lse, "lse"), _stream(stream)))
+    return out
 
 
 def dsa_mla_workspace_size(num_queries, H, d_v, k) -> int:

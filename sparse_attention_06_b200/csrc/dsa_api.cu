@@ -110,6 +110,8 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
+void set_last_error_message(const char* msg) { snprintf(g_msg, sizeof g_msg, "%s", msg); }
+
 bool encode_tmap_2d(void* tmap_out, const void* base, int elem_bytes, uint64_t inner,
                     uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
                     uint32_t box_outer, bool swizzle128) {

@@ -53,6 +53,9 @@ cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_
 int mla_tc_num_splits(int T, int k, int num_sms);
 size_t mla_tc_workspace_bytes(int T, int H, int d_v, int nsplit);
 
+// detail text returned by dsa_last_error_message() on this host thread
+void set_last_error_message(const char* msg);
+
 // tensor-map encoding through the driver entry point (no link-time libcuda dependency)
 bool encode_tmap_2d(void* tmap_out, const void* base, int elem_bytes, uint64_t inner,
                     uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
