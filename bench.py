@@ -488,7 +488,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="decode",
-                    choices=["tiny", "decode", "batched_decode", "prefill", "long_decode"])
+                    choices=["tiny", "decode", "batched_decode", "prefill", "long_decode", "profile_decode"])
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")

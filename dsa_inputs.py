@@ -231,12 +231,19 @@ def long_decode(B=16, L=202752, seed=0x5EED + 4) -> Spec:
                 q_pos=[L - 1] * B, key_dtype="e4m3", planted_frac=0.02, planted_sigma=3.0, seed=seed)
 
 
+def profile_decode(B=8, L=65536, seed=0x5EED + 5) -> Spec:
+    """bf16 decode, batch B at context L: a profiling case larger than L2 (0.75 GB resident)."""
+    return Spec("profile_decode_bf16_B%d_L%d" % (B, L), lens=[L] * B, q_req=list(range(B)),
+                q_pos=[L - 1] * B, seed=seed)
+
+
 WORKLOADS = {
     "tiny": tiny,
     "decode": decode,
     "batched_decode": batched_decode,
     "prefill": prefill,
     "long_decode": long_decode,
+    "profile_decode": profile_decode,
 }
 
 

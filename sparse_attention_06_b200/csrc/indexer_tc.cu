@@ -5,7 +5,10 @@
 //     score[t, s] = sum_h w[t,h] * ReLU(q[t,h,:] . khat[s,:])
 // with 64 indexer heads of 128 dims, bf16 queries, and bf16 keys or e4m3 keys with a per-token
 // scale (khat = code * scale; for scale > 0 the scale is applied after the head sum, which is the
-// same value).
+// same value).  bf16 keys multiply bf16 queries exactly as stored.  For e4m3 keys the product runs
+// in f16: every e4m3 code is exact in f16 (one conversion instruction per pair), and each query
+// tile is converted bf16 -> f16 once, which is exact for |q| in [2^-14, 65504] (smaller values
+// keep an absolute error below 2^-25).
 //
 // Shape of the computation: per tile of 128 consecutive key positions (two 64-token pages of the
 // paged key cache) one tensor-core product D[128 keys, 64*NQ] = K[128 keys, 128] . Q[64*NQ, 128]^T
@@ -18,7 +21,8 @@
 //   warp 0      TMA producer: key pages and query tiles into 128B-swizzled shared memory
 //   warp 1      TMEM allocation and the single thread that issues tcgen05.mma / tcgen05.commit
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator, ReLU, head sum, scale, score stores
-//   warps 6-9   (e4m3 keys only) dequantise the fp8 staging tile into the bf16 operand ring
+//   warps 6-9   (e4m3 keys only) convert the fp8 staging tile into the f16 operand ring and each
+//               query tile to f16 in place
 // Every wait is bounded (DSA_DEVERR_TIMEOUT); bad block ids and bad query metadata are flagged in
 // the device error word and skipped, never trapped.
 #include <cuda.h>
@@ -54,7 +58,7 @@ struct Cfg {
   static constexpr int OFF_Q = OFF_ST + STS * ST_BYTES;
   static constexpr int OFF_W = OFF_Q + QS * Q_BYTES;
   static constexpr int OFF_BAR = OFF_W + 4 * NQ * kHeads * 4;  // one copy of w per epilogue warp
-  static constexpr int NBAR = 2 * OPS + 2 * STS + 2 * QS + 4 + 1;
+  static constexpr int NBAR = 2 * OPS + 2 * STS + 3 * QS + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 64;
   static constexpr int SMEM = BYTES + 1024;  // slack for aligning the base
@@ -168,8 +172,8 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* 
   mbar_wait(bar, parity, err, nullptr);
 }
 
-// fp8 e4m3 x16 -> bf16 x16 (exact: every e4m3 value is a bf16 value)
-__device__ __forceinline__ void e4m3x16_to_bf16(const uint4& in, uint4& lo, uint4& hi) {
+// fp8 e4m3 x16 -> f16 x16 (exact: every e4m3 value is an f16 value)
+__device__ __forceinline__ void e4m3x16_to_f16(const uint4& in, uint4& lo, uint4& hi) {
   const uint32_t* w = reinterpret_cast<const uint32_t*>(&in);
   uint32_t outw[8];
 #pragma unroll
@@ -178,13 +182,25 @@ __device__ __forceinline__ void e4m3x16_to_bf16(const uint4& in, uint4& lo, uint
     for (int hpart = 0; hpart < 2; ++hpart) {
       const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * hpart)) & 0xFFFFu);
       const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
-      const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
-      outw[2 * i + hpart] = *reinterpret_cast<const uint32_t*>(&b);
+      outw[2 * i + hpart] = (uint32_t)h2.x | ((uint32_t)h2.y << 16);
     }
   }
   lo = make_uint4(outw[0], outw[1], outw[2], outw[3]);
   hi = make_uint4(outw[4], outw[5], outw[6], outw[7]);
+}
+
+// bf16 x8 -> f16 x8 in place (16 bytes)
+__device__ __forceinline__ uint4 bf16x8_to_f16(const uint4& in) {
+  uint4 out;
+  const uint32_t* a = reinterpret_cast<const uint32_t*>(&in);
+  uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a[i]));
+    const __half2 h = __float22half2_rn(f);
+    o[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return out;
 }
 
 template <int NQ, bool FP8>
@@ -205,7 +221,8 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
   uint64_t* st_empty = st_full + C::STS;
   uint64_t* q_full = st_empty + C::STS;
   uint64_t* q_empty = q_full + C::QS;
-  uint64_t* acc_full = q_empty + C::QS;
+  uint64_t* q_ready = q_empty + C::QS;  // (e4m3) query tile converted to f16
+  uint64_t* acc_full = q_ready + C::QS;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* mma_done = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -227,6 +244,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
     for (int i = 0; i < C::QS; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
+      mbar_init(&q_ready[i], 128);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -318,7 +336,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && lo < hi) {
-      const uint32_t idesc = idesc_f16(1u, 0u, 128u, (uint32_t)C::N);
+      const uint32_t idesc = idesc_f16(FP8 ? 0u : 1u, 0u, 128u, (uint32_t)C::N);  // f16 or bf16
       Walk<NQ> W;
       W.init(p, lo, hi);
       int grp, j, last = -1, m = -1, slot = -1;
@@ -330,7 +348,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
           last = grp;
           ++m;
           slot = m % C::QS;
-          if (!(ok = mbar_wait(&q_full[slot], (m / C::QS) & 1, p.err, abort_flag))) break;
+          if (!(ok = mbar_wait(FP8 ? &q_ready[slot] : &q_full[slot], (m / C::QS) & 1, p.err, abort_flag))) break;
         }
         const int s = (int)(i % C::OPS), use = (int)(i / C::OPS);
         if (!(ok = mbar_wait(&op_full[s], use & 1, p.err, abort_flag))) break;
@@ -362,28 +380,56 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
     const int quarter = warp & 3;              // TMEM lanes this warp may access
     const int r = quarter * 32 + lane;         // key row of the tile
     float* w_mine = w_s + (warp - 2) * NQ * kHeads;  // this warp's copy of the group's w
+    const int pg = r >> 6;                           // page of the tile holding this row
+    // Tiles are looked up ahead of their accumulator: the block id two tiles ahead and the e4m3
+    // scale one tile ahead, so that neither global load is waited on in the tile that issued it.
     Walk<NQ> W;
     W.init(p, lo, hi);
-    int grp, j, last = -1;
+    int g0 = -1, j0 = 0, g1 = -1, j1 = 0, g2 = -1, j2 = 0;
+    Group G0{0, 0, 0}, G1{0, 0, 0}, G2{0, 0, 0};
+    int b0 = -1, b1 = -1, b2 = -1;
+    float sc0 = 1.0f, sc1 = 1.0f;
+    if (W.next(p, g1, j1)) {
+      G1 = W.G;
+      b1 = page_block(p, G1, j1, pg, false);
+      if (W.next(p, g2, j2)) {
+        G2 = W.G;
+        b2 = page_block(p, G2, j2, pg, false);
+      } else {
+        g2 = -1;
+      }
+      if (FP8 && b1 >= 0) sc1 = p.key_scale[(int64_t)b1 * kPage + (r & 63)];
+    } else {
+      g1 = -1;
+    }
+    int last = -1;
     int npos[NQ];
     int64_t i = 0;
-    while (W.next(p, grp, j)) {
-      if (grp != last) {
+    while (g1 >= 0) {
+      // rotate: the tile to finish now is the one looked up last iteration
+      g0 = g1; j0 = j1; G0 = G1; b0 = b1; sc0 = sc1;
+      g1 = g2; j1 = j2; G1 = G2; b1 = b2;
+      sc1 = 1.0f;
+      if (g1 >= 0 && FP8 && b1 >= 0) sc1 = p.key_scale[(int64_t)b1 * kPage + (r & 63)];
+      if (g1 >= 0 && W.next(p, g2, j2)) {
+        G2 = W.G;
+        b2 = page_block(p, G2, j2, pg, false);
+      } else {
+        g2 = -1;
+      }
+      if (g0 != last) {
         __syncwarp();
-        for (int e = lane; e < NQ * kHeads; e += 32) w_mine[e] = p.w[(int64_t)grp * NQ * kHeads + e];
+        for (int e = lane; e < NQ * kHeads; e += 32) w_mine[e] = p.w[(int64_t)g0 * NQ * kHeads + e];
         __syncwarp();
 #pragma unroll
-        for (int qi = 0; qi < NQ; ++qi) npos[qi] = p.q_pos[grp * NQ + qi] + 1;
-        last = grp;
+        for (int qi = 0; qi < NQ; ++qi) npos[qi] = p.q_pos[g0 * NQ + qi] + 1;
+        last = g0;
       }
       const int a = (int)(i & 1), use = (int)(i >> 1);
       if (!warp_wait(&acc_full[a], use & 1, p.err, abort_flag)) break;
       tc_fence_after();
-      const int pg = r >> 6;
-      const int blk = page_block(p, W.G, j, pg, false);
-      const int s = j * kTileKeys + r;
-      float scale = 1.0f;
-      if (FP8 && blk >= 0) scale = p.key_scale[(int64_t)blk * kPage + (r & 63)];
+      const int s = j0 * kTileKeys + r;
+      const float scale = FP8 ? sc0 : 1.0f;
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * C::N);
 #pragma unroll
       for (int qi = 0; qi < NQ; ++qi) {
@@ -403,7 +449,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
           acc0 = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * h4 + 2]), 0.0f), acc0);
           acc1 = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * h4 + 3]), 0.0f), acc1);
         }
-        if (blk >= 0 && s < npos[qi]) p.scores[(int64_t)(grp * NQ + qi) * p.ld + s] = (acc0 + acc1) * scale;
+        if (b0 >= 0 && s < npos[qi]) p.scores[(int64_t)(g0 * NQ + qi) * p.ld + s] = (acc0 + acc1) * scale;
       }
       tc_fence_before();
       __syncwarp();
@@ -415,9 +461,21 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
     const int ct = tid - 192;  // 0..127
     Walk<NQ> W;
     W.init(p, lo, hi);
-    int grp, j;
+    int grp, j, last = -1, m = -1;
     int64_t i = 0;
     while (W.next(p, grp, j)) {
+      if (grp != last) {
+        // a new query tile: convert it to f16 in place once it has landed
+        last = grp;
+        ++m;
+        const int slot = m % C::QS;
+        if (!warp_wait(&q_full[slot], (m / C::QS) & 1, p.err, abort_flag)) break;
+        uint8_t* q = q_slots + slot * C::Q_BYTES;
+        for (int off = ct * 16; off < C::Q_BYTES; off += 128 * 16)
+          *reinterpret_cast<uint4*>(q + off) = bf16x8_to_f16(*reinterpret_cast<const uint4*>(q + off));
+        fence_proxy_async_smem();
+        mbar_arrive(&q_ready[slot]);
+      }
       const int s8 = (int)(i % C::STS), u8 = (int)(i / C::STS);
       if (!warp_wait(&st_full[s8], u8 & 1, p.err, abort_flag)) break;
       const int so = (int)(i % C::OPS), uo = (int)(i / C::OPS);
@@ -430,7 +488,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
         const int row = piece >> 3, c = piece & 7;
         const uint4 in = *reinterpret_cast<const uint4*>(src + row * 128 + c * 16);
         uint4 lo4, hi4;
-        e4m3x16_to_bf16(in, lo4, hi4);
+        e4m3x16_to_f16(in, lo4, hi4);
         uint8_t* chunk = dst + (c >> 2) * C::CHUNK_BYTES;
         const uint32_t p0 = (uint32_t)((c & 3) * 2);
         *reinterpret_cast<uint4*>(chunk + sw128_offset(row, p0)) = lo4;

@@ -46,8 +46,9 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + Q_BYTES;
 constexpr int OFF_P = OFF_K + 2 * K_BYTES;
 constexpr int OFF_BAR = OFF_P + P_BYTES;
-constexpr int NBAR = 13;
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int NBAR = 15;
+constexpr int OFF_MASK = OFF_BAR + NBAR * 8;   // valid-row masks: 2 stages x 2 gather warps
+constexpr int OFF_MISC = OFF_MASK + 16;
 constexpr int BYTES = OFF_MISC + 32;
 constexpr int SMEM = BYTES + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
@@ -85,14 +86,16 @@ __device__ __forceinline__ void unit_coords(const Params& p, int u, int& t, int&
   sp = ts % p.nsplit;
 }
 
-// Physical pool row of selection slot `slot` of query t (request req, position pos), or -1 when
-// the slot is past the split / the selection, holds -1, or is out of range (flagged when
-// `report`).  The gather warps and the softmax warps apply the same rule.
-__device__ __forceinline__ int64_t slot_row(const Params& p, int t, int req, int pos, bool qok, int sp,
-                                            int slot, bool report) {
-  if (!qok || slot >= min(p.k, (sp + 1) * p.ks)) return -1;
-  const int ps = p.idx[(int64_t)t * p.k + slot];
-  if (ps == -1) return -1;
+// Row lookup of selection slot `slot` of query t in two halves, so that the dependent loads
+// can be issued a tile apart: the selected position of a slot (kNoSlot when the slot is outside the split or the selection) ...
+constexpr int kNoSlot = -2;
+__device__ __forceinline__ int slot_pos(const Params& p, int t, bool qok, int sp, int slot) {
+  if (!qok || slot >= min(p.k, (sp + 1) * p.ks)) return kNoSlot;
+  return p.idx[(int64_t)t * p.k + slot];
+}
+// ... and the physical block holding it (-1 when unused or out of range; flagged when `report`).
+__device__ __forceinline__ int pos_block(const Params& p, int req, int pos, int ps, bool report) {
+  if (ps == kNoSlot || ps == -1) return -1;
   if (ps < 0 || ps > pos) {
     if (report) raise_error(p.err, DSA_DEVERR_INDEX);
     return -1;
@@ -103,7 +106,7 @@ __device__ __forceinline__ int64_t slot_row(const Params& p, int t, int req, int
     if (report) raise_error(p.err, DSA_DEVERR_BLOCK_ID);
     return -1;
   }
-  return (int64_t)blk * kPage + (ps % kPage);
+  return blk;
 }
 
 __device__ __forceinline__ int unit_tiles(const Params& p, int sp) {
@@ -129,6 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = bars + 10;
   uint64_t* pv_done = bars + 11;
   uint64_t* mma_fin = bars + 12;
+  uint64_t* m_full = bars + 13;  // [2] valid-row mask of a stage published
+  uint32_t* masks = reinterpret_cast<uint32_t*>(smem + OFF_MASK);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 8);
 
@@ -147,6 +152,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
     mbar_init(mma_fin, 1);
+    mbar_init(&m_full[0], 2);
+    mbar_init(&m_full[1], 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -180,12 +187,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const int ntiles = unit_tiles(p, sp);
+      // Row lookups of this warp's 16 keys per tile (lanes 0..15), software-pipelined so that no
+      // load is waited on in the tile it is issued: the selected position two tiles ahead and the
+      // block id one tile ahead.
+      const bool mine = lane < 16;
+      const int kslot = sp * p.ks + gw * 16 + lane;
+      int ps_j = mine && ntiles > 0 ? slot_pos(p, t, qok, sp, kslot) : kNoSlot;
+      int ps_j1 = mine && ntiles > 1 ? slot_pos(p, t, qok, sp, kslot + kTile) : kNoSlot;
+      int blk_j = mine ? pos_block(p, req, pos, ps_j, v == 0) : -1;
       for (int j = 0; j < ntiles; ++j, ++gi) {
         const int s = gi & 1;
+        const int64_t row = blk_j >= 0 ? (int64_t)blk_j * kPage + (ps_j % kPage) : -1;
+        const int blk_j1 = mine && j + 1 < ntiles ? pos_block(p, req, pos, ps_j1, v == 0) : -1;
+        const int ps_j2 = mine && j + 2 < ntiles ? slot_pos(p, t, qok, sp, kslot + (j + 2) * kTile) : kNoSlot;
         if (gi >= 2 && !(ok = warp_wait(&k_empty[s], ((gi >> 1) - 1) & 1, p.err, abort_flag))) break;
-        // row of each of this warp's 16 keys: lanes 0..15 look theirs up
-        const int slot = sp * p.ks + j * kTile + gw * 16 + lane;
-        const int64_t row = lane < 16 ? slot_row(p, t, req, pos, qok, sp, slot, v == 0) : -1;
+        // publish which rows of the tile are real to the softmax warps
+        const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, row >= 0) & 0xFFFFu;
+        if (lane == 0) {
+          masks[s * 2 + gw] = vmask;
+          mbar_arrive(&m_full[s]);
+        }
+        ps_j = ps_j1;
+        ps_j1 = ps_j2;
+        blk_j = blk_j1;
         uint8_t* stage = k_ring + s * K_BYTES;
         const uint32_t stage_u32 = smem_u32(stage);
 #pragma unroll 1
@@ -281,13 +305,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int t, sp, v;
       unit_coords(p, u, t, sp, v);
       const int ntiles = unit_tiles(p, sp);
-      const int req = p.q_req[t];
-      const int pos = p.q_pos[t];
-      const bool qok = req >= 0 && req < p.num_reqs && pos >= 0 && pos < p.max_context;
       float m_used = -INFINITY, l = 0.0f;
       for (int j = 0; j < ntiles; ++j) {
         const int g = gi + j, s = g & 1;
         if (!(ok = warp_wait(&s_full[s], (g >> 1) & 1, p.err, abort_flag))) break;
+        if (!(ok = warp_wait(&m_full[s], (g >> 1) & 1, p.err, abort_flag))) break;
         tc_fence_after();
         uint32_t sv[32];
         tmem_ld16(lane_base + TM_S + s * kTile, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
@@ -296,8 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[s]);
-        const uint32_t valid =
-            __ballot_sync(0xFFFFFFFFu, slot_row(p, t, req, pos, qok, sp, sp * p.ks + j * kTile + lane, false) >= 0);
+        const uint32_t valid = masks[s * 2 + 0] | (masks[s * 2 + 1] << 16);
         float x[32];
         float mt = -INFINITY;
 #pragma unroll
@@ -361,48 +382,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv = l > 0.0f ? 1.0f / l : 0.0f;
       const float lse = l > 0.0f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
       const int64_t orow = (int64_t)t * kH + r;
-      if (p.nsplit == 1) {
-        __nv_bfloat16* dst = p.out + orow * kDv + v * kHalf;
+      // O / l in 64-column pieces: four TMEM loads in flight per wait, then the stores
+      const int64_t prow = ((int64_t)t * p.nsplit + sp) * kH + r;
 #pragma unroll 1
-        for (int c0 = 0; c0 < kHalf; c0 += 16) {
-          uint32_t o[16];
-          if (ntiles > 0) {
-            tmem_ld16(lane_base + TM_O + c0, o);
-            tmem_wait_ld();
-          }
-          uint32_t pk[8];
+      for (int c0 = 0; c0 < kHalf; c0 += 64) {
+        uint32_t o[64];
+        if (ntiles > 0) {
+          tmem_ld16(lane_base + TM_O + c0, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+          tmem_ld16(lane_base + TM_O + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
+          tmem_ld16(lane_base + TM_O + c0 + 32, *reinterpret_cast<uint32_t(*)[16]>(&o[32]));
+          tmem_ld16(lane_base + TM_O + c0 + 48, *reinterpret_cast<uint32_t(*)[16]>(&o[48]));
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-          for (int c = 0; c < 16; c += 2) {
-            const float a = ntiles > 0 ? __uint_as_float(o[c]) * inv : 0.0f;
-            const float b = ntiles > 0 ? __uint_as_float(o[c + 1]) * inv : 0.0f;
-            const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-            pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&h);
-          }
-          *reinterpret_cast<uint4*>(dst + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(dst + c0 + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          for (int c = 0; c < 64; ++c) o[c] = 0u;
         }
-        if (v == 0 && p.lse) p.lse[orow] = lse;
-      } else {
-        const int64_t prow = ((int64_t)t * p.nsplit + sp) * kH + r;
-        float* dst = p.part_o + prow * kDv + v * kHalf;
-#pragma unroll 1
-        for (int c0 = 0; c0 < kHalf; c0 += 16) {
-          uint32_t o[16];
-          if (ntiles > 0) {
-            tmem_ld16(lane_base + TM_O + c0, o);
-            tmem_wait_ld();
-          }
+        if (p.nsplit == 1) {
+          __nv_bfloat16* dst = p.out + orow * kDv + v * kHalf + c0;
 #pragma unroll
-          for (int c = 0; c < 16; c += 4) {
-            float4 f;
-            f.x = ntiles > 0 ? __uint_as_float(o[c]) * inv : 0.0f;
-            f.y = ntiles > 0 ? __uint_as_float(o[c + 1]) * inv : 0.0f;
-            f.z = ntiles > 0 ? __uint_as_float(o[c + 2]) * inv : 0.0f;
-            f.w = ntiles > 0 ? __uint_as_float(o[c + 3]) * inv : 0.0f;
-            *reinterpret_cast<float4*>(dst + c0 + c) = f;
+          for (int c = 0; c < 64; c += 8) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(o[c + e]) * inv, __uint_as_float(o[c + e + 1]) * inv);
+              pk[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            *reinterpret_cast<uint4*>(dst + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
+        } else {
+          float* dst = p.part_o + prow * kDv + v * kHalf + c0;
+#pragma unroll
+          for (int c = 0; c < 64; c += 4)
+            *reinterpret_cast<float4*>(dst + c) = make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
+                                                              __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
         }
-        if (v == 0) p.part_lse[prow] = lse;
+      }
+      if (v == 0) {
+        if (p.nsplit == 1) {
+          if (p.lse) p.lse[orow] = lse;
+        } else {
+          p.part_lse[prow] = lse;
+        }
       }
       tc_fence_before();
     }
@@ -417,44 +437,60 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // grid (T, 128 heads), block 128: merge the split partials of one (query, head) row; each thread
-// owns 4 of the 512 value columns.
+// owns 4 of the 512 value columns.  The split weights exp(LSE_sp - max) are computed once into
+// shared memory, so the per-split loads of the accumulation loop are independent.
+constexpr int kMaxSplits = 64;
 __global__ void __launch_bounds__(128) mla_combine_kernel(const float* __restrict__ part_o,
                                                           const float* __restrict__ part_lse, int nsplit,
                                                           __nv_bfloat16* __restrict__ out,
                                                           float* __restrict__ lse_out) {
+  __shared__ float wts[kMaxSplits];
+  __shared__ float s_mx, s_inv, s_lse;
   const int t = blockIdx.x, h = blockIdx.y, c = threadIdx.x * 4;
   const int64_t row0 = (int64_t)t * nsplit * kH + h;  // partial row of split 0; split sp adds sp*kH
-  float mx = -INFINITY;
-  for (int sp = 0; sp < nsplit; ++sp) mx = fmaxf(mx, part_lse[row0 + (int64_t)sp * kH]);
-  float wsum = 0.0f;
+  if (threadIdx.x < 32) {
+    float mx = -INFINITY;
+    for (int sp = threadIdx.x; sp < nsplit; sp += 32) mx = fmaxf(mx, part_lse[row0 + (int64_t)sp * kH]);
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    float sum = 0.0f;
+    for (int sp = threadIdx.x; sp < nsplit; sp += 32) {
+      const float ls = part_lse[row0 + (int64_t)sp * kH];
+      const float wgt = ls == -INFINITY ? 0.0f : expf(ls - mx);
+      wts[sp] = wgt;
+      sum += wgt;
+    }
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+    if (threadIdx.x == 0) {
+      s_inv = sum > 0.0f ? 1.0f / sum : 0.0f;
+      s_lse = sum > 0.0f ? mx + logf(sum) : -INFINITY;
+    }
+  }
+  __syncthreads();
   float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll 8
   for (int sp = 0; sp < nsplit; ++sp) {
-    const int64_t prow = row0 + (int64_t)sp * kH;
-    const float ls = part_lse[prow];
-    if (ls == -INFINITY) continue;
-    const float wgt = expf(ls - mx);
-    wsum += wgt;
-    const float4 a = *reinterpret_cast<const float4*>(part_o + prow * kDv + c);
+    const float wgt = wts[sp];
+    const float4 a = __ldg(reinterpret_cast<const float4*>(part_o + (row0 + (int64_t)sp * kH) * kDv + c));
     acc.x = fmaf(wgt, a.x, acc.x);
     acc.y = fmaf(wgt, a.y, acc.y);
     acc.z = fmaf(wgt, a.z, acc.z);
     acc.w = fmaf(wgt, a.w, acc.w);
   }
-  const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
+  const float inv = s_inv;
   const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
   const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
   uint2 pk;
   pk.x = *reinterpret_cast<const uint32_t*>(&lo);
   pk.y = *reinterpret_cast<const uint32_t*>(&hi);
   *reinterpret_cast<uint2*>(out + ((int64_t)t * kH + h) * kDv + c) = pk;
-  if (lse_out && threadIdx.x == 0) lse_out[(int64_t)t * kH + h] = wsum > 0.0f ? mx + logf(wsum) : -INFINITY;
+  if (lse_out && threadIdx.x == 0) lse_out[(int64_t)t * kH + h] = s_lse;
 }
 
 int splits_for(int T, int k, int num_sms) {
   const int tiles_q = (k + kTile - 1) / kTile;  // tiles per (query, half)
   const double ideal = 2.0 * T * tiles_q / num_sms;
   int best = 1;
-  for (int n = 1; n <= 64; n *= 2) {
+  for (int n = 1; n <= kMaxSplits; n *= 2) {
     int ks = ((k + n - 1) / n + kTile - 1) / kTile * kTile;
     if (ks < 2 * kTile && n > 1) break;
     const int ns = (k + ks - 1) / ks;

@@ -5,14 +5,22 @@
 // sees fewer than K positions keeps all of them.  Ties go to the lower position, and the chosen
 // positions are emitted in ascending order, so the result is unique and deterministic.
 //
-// Method (one CTA of 1024 threads per query row):
-//   1. every score is mapped to an order-preserving 32-bit key (larger score -> larger key,
-//      -0.0 folded onto +0.0, NaN -> lowest key plus an error bit);
-//   2. three radix passes (11 + 11 + 10 bits, shared-memory histograms) find the exact key value
-//      Tk of the K-th largest element and how many elements equal to Tk must be taken (need);
-//   3. one in-order pass over the row takes every key > Tk and the first `need` keys == Tk,
-//      using block-wide prefix counts, and writes their positions in ascending order.
-// All counts are order-independent, so the result does not depend on atomic ordering.
+// Scores are compared through an order-preserving 32-bit key (larger score -> larger key, -0.0
+// folded onto +0.0, NaN -> the lowest key and an error bit).  One CTA of 1024 threads per row:
+//
+// Fast path (rows up to 262144 positions):
+//   1. sample one 32-score chunk out of every 32 and radix-select from the sample a threshold tau
+//      expected to leave ~1.5 K scores at or above it;
+//   2. one pass over the row appends every (key, position) with key >= tau to shared memory
+//      (warp-aggregated);
+//   3. if at least K and at most kCap scores were collected, the exact K-th key Tk among them is
+//      found by radix select (every score >= Tk is a candidate, so it is the row's K-th key), the
+//      keys > Tk are marked in a position bitmap, and of the keys == Tk the lowest positions are
+//      marked (a radix select on the positions);
+//   4. a prefix sum of the bitmap's popcounts writes the marked positions in ascending order.
+// Exact path (otherwise): three radix passes over the row find Tk and the number of ties to
+// take, and one in-order pass with block-wide prefix counts writes the positions.
+// Every count is order-independent, so the result does not depend on the order of atomics.
 #include "common.cuh"
 #include "internal.h"
 
@@ -23,6 +31,20 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
+constexpr int kCap = 8192;            // candidate capacity of the fast path
+constexpr int kMaxRow = 262144;       // bitmap capacity (positions) of the fast path
+constexpr int kChunk = 32;            // sampled chunk length
+constexpr int kSampleEvery = 32;      // one chunk of every kSampleEvery
+
+struct Smem {
+  uint32_t hist[kBins];
+  uint32_t warp_tot[kWarps + 1];
+  uint32_t scal[8];
+  uint32_t sample[kCap];    // sample keys, later the positions of the tied candidates
+  uint32_t cand_key[kCap];
+  uint32_t cand_pos[kCap];
+  uint32_t bitmap[kMaxRow / 32];
+};
 
 __device__ __forceinline__ uint32_t order_key(float f, bool& is_nan) {
   uint32_t u = __float_as_uint(f);
@@ -35,8 +57,7 @@ __device__ __forceinline__ uint32_t order_key(float f, bool& is_nan) {
 }
 
 // Exclusive prefix sum of `v` over the block; returns the prefix, writes the block total.
-__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_tot,
-                                                         uint32_t& total) {
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_tot, uint32_t& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t incl = v;
 #pragma unroll
@@ -54,8 +75,8 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
       uint32_t y = __shfl_up_sync(0xFFFFFFFFu, wi, o);
       if (lane >= o) wi += y;
     }
-    if (lane < kWarps) warp_tot[lane] = wi - wv;  // exclusive warp offsets
-    if (lane == 31) warp_tot[kWarps] = wi;        // block total
+    if (lane < kWarps) warp_tot[lane] = wi - wv;
+    if (lane == 31) warp_tot[kWarps] = wi;
   }
   __syncthreads();
   uint32_t res = warp_tot[warp] + incl - v;
@@ -64,100 +85,248 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
   return res;
 }
 
-__global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict__ scores,
-                                                        int64_t ld, const int32_t* __restrict__ q_pos,
-                                                        int k, int32_t* __restrict__ idx, int* err) {
-  __shared__ uint32_t hist[kBins];
-  __shared__ uint32_t warp_tot[kWarps + 1];
-  __shared__ uint32_t s_digit, s_above;
-  __shared__ int s_nan;
-
-  const int t = blockIdx.x;
-  int64_t n = (int64_t)q_pos[t] + 1;
-  if (n > ld) {  // a row cannot hold more scores than its stride
-    if (threadIdx.x == 0) raise_error(err, DSA_DEVERR_REQUEST);
-    n = ld;
+// After a histogram pass over nbins (1024 or 2048) bins: find the digit holding the krem-th
+// largest counted key; writes the digit and the count of keys in higher digits to S.scal[0..1].
+// Thread i owns the bins nbins-1-2i and nbins-2-2i (from the top), a block-wide prefix sum gives
+// the count above each pair, and the one thread whose pair holds the krem-th key resolves it.
+__device__ __forceinline__ void find_digit(Smem& S, int nbins, uint32_t krem) {
+  const int per = nbins / kThreads;  // 1 or 2 bins per thread
+  const int top = nbins - 1 - per * threadIdx.x;
+  uint32_t h0 = S.hist[top];
+  uint32_t h1 = per == 2 ? S.hist[top - 1] : 0u;
+  uint32_t tot;
+  const uint32_t above = block_exclusive_scan(h0 + h1, S.warp_tot, tot);
+  if (above < krem && krem <= above + h0 + h1) {
+    if (krem <= above + h0) {
+      S.scal[0] = (uint32_t)top;
+      S.scal[1] = above;
+    } else {
+      S.scal[0] = (uint32_t)(top - 1);
+      S.scal[1] = above + h0;
+    }
   }
-  int32_t* out = idx + (int64_t)t * k;
-  if (n <= k) {
-    for (int j = threadIdx.x; j < k; j += kThreads) out[j] = j < n ? j : -1;
-    return;
-  }
-  const float* row = scores + (int64_t)t * ld;
-  if (threadIdx.x == 0) s_nan = 0;
+}
 
-  uint32_t prefix = 0u, hmask = 0u, krem = (uint32_t)k;
+// Radix select over keys produced by `get(i)` for i in [0, m): the value of the j-th largest
+// (1-based) and the number of keys strictly greater.  Block-wide; every thread gets the result.
+template <class Get>
+__device__ void radix_select(Smem& S, int64_t m, uint32_t j, Get get, uint32_t& value, uint32_t& above) {
+  uint32_t prefix = 0u, hmask = 0u, krem = j;
   const int shifts[3] = {21, 10, 0};
   const int widths[3] = {11, 11, 10};
-  bool saw_nan = false;
+#pragma unroll 1
   for (int pass = 0; pass < 3; ++pass) {
     const int shift = shifts[pass];
     const uint32_t dmask = (1u << widths[pass]) - 1u;
-    const int nbins = 1 << widths[pass];
-    for (int b = threadIdx.x; b < kBins; b += kThreads) hist[b] = 0u;
+    for (int b = threadIdx.x; b < kBins; b += kThreads) S.hist[b] = 0u;
     __syncthreads();
-    for (int64_t i = threadIdx.x; i < n; i += kThreads) {
-      uint32_t key = order_key(row[i], saw_nan);
-      if ((key & hmask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+    // lanes of a warp that hit the same bin add together (scores share their top bits)
+    for (int64_t i0 = 0; i0 < m; i0 += kThreads) {
+      const int64_t i = i0 + threadIdx.x;
+      uint32_t key = 0u;
+      bool in = false;
+      if (i < m) {
+        key = get(i);
+        in = (key & hmask) == prefix;
+      }
+      const uint32_t bin = in ? ((key >> shift) & dmask) : 0xFFFFFFFFu;
+      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+      if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&S.hist[bin], (uint32_t)__popc(peers));
     }
     __syncthreads();
-    if (threadIdx.x < 32) {
-      // lane L owns bins [L*per, (L+1)*per); find the digit holding the krem-th largest key
-      const int lane = threadIdx.x;
-      const int per = nbins / 32;
-      uint32_t mine = 0u;
-      for (int b = 0; b < per; ++b) mine += hist[lane * per + b];
-      // suffix sums over lanes (bins above and including lane L)
-      uint32_t suf = mine;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_down_sync(0xFFFFFFFFu, suf, o);
-        if (lane + o < 32) suf += y;
-      }
-      const uint32_t above_lane = suf - mine;  // bins of higher lanes
-      const bool hit = suf >= krem && above_lane < krem;
-      const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, hit);
-      if (hit && lane == 31 - __clz(ballot)) {
-        uint32_t run = above_lane;
-        for (int b = per - 1; b >= 0; --b) {
-          const uint32_t h = hist[lane * per + b];
-          if (run + h >= krem) {
-            s_digit = (uint32_t)(lane * per + b);
-            s_above = run;
-            break;
-          }
-          run += h;
-        }
-      }
-    }
+    find_digit(S, 1 << widths[pass], krem);
     __syncthreads();
-    prefix |= s_digit << shift;
+    prefix |= S.scal[0] << shift;
     hmask |= dmask << shift;
-    krem -= s_above;
+    krem -= S.scal[1];
     __syncthreads();
   }
-  if (saw_nan) s_nan = 1;  // benign race: every writer stores 1
-  const uint32_t tk = prefix;
-  const uint32_t need = krem;  // number of keys equal to tk to take, lowest positions first
+  value = prefix;
+  above = j - krem;
+}
 
+// Exact path: radix select over the row in global memory, then one in-order pass.
+__device__ void topk_exact(Smem& S, const float* row, int64_t n, int k, int32_t* out, bool& saw_nan) {
+  uint32_t tk, above;
+  radix_select(S, n, (uint32_t)k, [&](int64_t i) { return order_key(row[i], saw_nan); }, tk, above);
+  const uint32_t need = (uint32_t)k - above;  // keys equal to tk to take, lowest positions first
   uint32_t base = 0u, eq_seen = 0u;
   for (int64_t c0 = 0; c0 < n; c0 += kThreads) {
     const int64_t i = c0 + threadIdx.x;
     bool dummy = false;
-    const uint32_t key = i < n ? order_key(row[i], dummy) : 0u;
     const bool valid = i < n;
+    const uint32_t key = valid ? order_key(row[i], dummy) : 0u;
     const uint32_t eq = (valid && key == tk) ? 1u : 0u;
     uint32_t eq_tot;
-    const uint32_t eq_rank = block_exclusive_scan(eq, warp_tot, eq_tot);
+    const uint32_t eq_rank = block_exclusive_scan(eq, S.warp_tot, eq_tot);
     const uint32_t take = (valid && (key > tk || (eq && eq_seen + eq_rank < need))) ? 1u : 0u;
     uint32_t take_tot;
-    const uint32_t at = block_exclusive_scan(take, warp_tot, take_tot);
+    const uint32_t at = block_exclusive_scan(take, S.warp_tot, take_tot);
     if (take && base + at < (uint32_t)k) out[base + at] = (int32_t)i;
     base += take_tot;
     eq_seen += eq_tot;
   }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    topk_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ q_pos, int k,
+                int32_t* __restrict__ idx, int* err) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  Smem& S = *reinterpret_cast<Smem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int t = blockIdx.x;
+  int64_t n = (int64_t)q_pos[t] + 1;
+  if (n > ld) {  // a row cannot hold more scores than its stride
+    if (tid == 0) raise_error(err, DSA_DEVERR_REQUEST);
+    n = ld;
+  }
+  int32_t* out = idx + (int64_t)t * k;
+  if (n <= k) {
+    for (int j = tid; j < k; j += kThreads) out[j] = j < n ? j : -1;
+    return;
+  }
+  const float* row = scores + (int64_t)t * ld;
+  bool saw_nan = false;
+  if (tid == 0) {
+    S.scal[2] = 0u;  // candidate count
+    S.scal[3] = 0u;  // tie count
+    S.scal[4] = 0u;  // NaN seen
+  }
+
+  bool fast = n <= kMaxRow;
+  if (fast) {
+    // 1. threshold from a chunked sample (or take every score when the row fits the buffer)
+    uint32_t tau = 0u;
+    if (n > kCap) {
+      const int64_t full = n / (kChunk * kSampleEvery);
+      const int64_t rest = n % (kChunk * kSampleEvery);
+      const int ns = (int)(full * kChunk + (rest < kChunk ? rest : kChunk));
+      for (int s = tid; s < ns; s += kThreads) {
+        const int64_t i = (int64_t)(s / kChunk) * (kChunk * kSampleEvery) + (s % kChunk);
+        S.sample[s] = order_key(row[i], saw_nan);
+      }
+      __syncthreads();
+      // rank in the sample whose key should leave ~1.5 K scores of the row at or above it
+      const double frac = (double)ns / (double)n;
+      int64_t js = (int64_t)(1.5 * k * frac) + 8;
+      if (js > ns) js = ns;
+      uint32_t above_s;
+      radix_select(S, ns, (uint32_t)js, [&](int64_t i) { return S.sample[i]; }, tau, above_s);
+    }
+    __syncthreads();
+    // 2. collect every score at or above tau.  The row is read in 16-score groups per thread
+    //    (four 16-byte loads when the row is 16-byte aligned), and the next group's loads are
+    //    issued before the current group is appended, so that a load is always in flight.
+    const bool vec = ((reinterpret_cast<uintptr_t>(row) & 15u) == 0);
+    constexpr int kPer = 16;                       // scores per thread per step
+    const int64_t step = (int64_t)kPer * kThreads;
+    float cur[kPer], nxt[kPer];
+    auto load_group = [&](int64_t base, float (&v)[kPer]) {
+      if (vec && base + step <= n) {
+#pragma unroll
+        for (int u = 0; u < kPer / 4; ++u) {
+          const float4 f = __ldg(reinterpret_cast<const float4*>(row + base + (int64_t)(u * kThreads + tid) * 4));
+          v[4 * u] = f.x; v[4 * u + 1] = f.y; v[4 * u + 2] = f.z; v[4 * u + 3] = f.w;
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < kPer / 4; ++u) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int64_t i = base + (int64_t)(u * kThreads + tid) * 4 + e;
+            v[4 * u + e] = i < n ? row[i] : __int_as_float(0x7FC00000);  // NaN marks "past the row"
+          }
+        }
+      }
+    };
+    if (n > 0) load_group(0, cur);
+    for (int64_t base = 0; base < n; base += step) {
+      if (base + step < n) load_group(base + step, nxt);
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int64_t i = base + (int64_t)((u >> 2) * kThreads + tid) * 4 + (u & 3);
+        bool pred = false;
+        uint32_t key = 0u;
+        if (i < n) {
+          key = order_key(cur[u], saw_nan);
+          pred = key >= tau;
+        }
+        const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, pred);
+        if (ballot) {
+          const int leader = __ffs(ballot) - 1;
+          uint32_t b0 = 0u;
+          if (lane == leader) b0 = atomicAdd(&S.scal[2], (uint32_t)__popc(ballot));
+          b0 = __shfl_sync(0xFFFFFFFFu, b0, leader);
+          if (pred) {
+            const uint32_t pos = b0 + __popc(ballot & ((1u << lane) - 1u));
+            if (pos < kCap) {
+              S.cand_key[pos] = key;
+              S.cand_pos[pos] = (uint32_t)i;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) cur[u] = nxt[u];
+    }
+    __syncthreads();
+    const uint32_t m = S.scal[2];
+    fast = m >= (uint32_t)k && m <= (uint32_t)kCap;
+    if (fast) {
+      // 3. exact K-th key among the candidates, then mark the selection in the bitmap
+      uint32_t tk, above;
+      radix_select(S, m, (uint32_t)k, [&](int64_t i) { return S.cand_key[i]; }, tk, above);
+      const uint32_t need = (uint32_t)k - above;
+      const int words = (int)((n + 31) / 32);
+      for (int w = tid; w < words; w += kThreads) S.bitmap[w] = 0u;
+      __syncthreads();
+      for (uint32_t c = tid; c < m; c += kThreads) {
+        const uint32_t key = S.cand_key[c];
+        const uint32_t pos = S.cand_pos[c];
+        if (key > tk) {
+          atomicOr(&S.bitmap[pos >> 5], 1u << (pos & 31));
+        } else if (key == tk) {
+          const uint32_t e = atomicAdd(&S.scal[3], 1u);
+          S.sample[e] = pos;
+        }
+      }
+      __syncthreads();
+      const uint32_t neq = S.scal[3];
+      uint32_t pos_cut = 0xFFFFFFFFu;  // take tied positions <= pos_cut
+      if (neq > need) {
+        // the `need` lowest positions among the ties: radix select on the complemented position
+        uint32_t v, ab;
+        radix_select(S, neq, need, [&](int64_t i) { return ~S.sample[i]; }, v, ab);
+        pos_cut = ~v;
+      }
+      for (uint32_t e = tid; e < neq; e += kThreads) {
+        const uint32_t pos = S.sample[e];
+        if (pos <= pos_cut) atomicOr(&S.bitmap[pos >> 5], 1u << (pos & 31));
+      }
+      __syncthreads();
+      // 4. ascending output: prefix sum of per-thread popcounts over contiguous word ranges
+      const int wpt = (words + kThreads - 1) / kThreads;
+      const int w0 = tid * wpt;
+      const int w1 = min(words, w0 + wpt);
+      uint32_t cnt = 0u;
+      for (int w = w0; w < w1; ++w) cnt += (uint32_t)__popc(S.bitmap[w]);
+      uint32_t total;
+      uint32_t at = block_exclusive_scan(cnt, S.warp_tot, total);
+      for (int w = w0; w < w1; ++w) {
+        uint32_t bits = S.bitmap[w];
+        while (bits) {
+          const int b = __ffs(bits) - 1;
+          bits &= bits - 1u;
+          if (at < (uint32_t)k) out[at] = w * 32 + b;
+          ++at;
+        }
+      }
+    }
+  }
+  if (!fast) topk_exact(S, row, n, k, out, saw_nan);
+  if (saw_nan) S.scal[4] = 1u;  // benign race: every writer stores 1
   __syncthreads();
-  if (threadIdx.x == 0 && s_nan) raise_error(err, DSA_DEVERR_NAN_SCORE);
+  if (tid == 0 && S.scal[4]) raise_error(err, DSA_DEVERR_NAN_SCORE);
 }
 
 }  // namespace
@@ -165,7 +334,10 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, int T, int k,
                         int32_t* idx, int* err, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  topk_kernel<<<T, kThreads, 0, s>>>(scores, ld, q_pos, k, idx, err);
+  const int smem = (int)sizeof(Smem);
+  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  topk_kernel<<<T, kThreads, smem, s>>>(scores, ld, q_pos, k, idx, err);
   return cudaGetLastError();
 }
 
