@@ -355,18 +355,20 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
         const int a = (int)(i & 1), ause = (int)(i >> 1);
         if (ause >= 1 && !(ok = mbar_wait(&acc_empty[a], (ause - 1) & 1, p.err, abort_flag))) break;
         tc_fence_after();
-        const uint32_t a_base = smem_u32(op_ring + s * C::OP_BYTES);
-        const uint32_t b_base = smem_u32(q_slots + slot * C::Q_BYTES);
+        // 8 MMAs of K = 16: two 64-dim column blocks, four K steps of 32 bytes each (the
+        // descriptor's start-address field counts 16-byte units)
+        const uint64_t ad = sw128_desc(smem_u32(op_ring + s * C::OP_BYTES), 16, 1024);
+        const uint64_t bd = sw128_desc(smem_u32(q_slots + slot * C::Q_BYTES), 16, 1024);
         const uint32_t d = tmem_base + (uint32_t)(a * C::N);
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = sw128_desc(a_base + c * C::CHUNK_BYTES + k * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(b_base + c * C::Q_CHUNK + k * 32, 16, 1024);
-            mma_f16_ss(d, ad, bd, idesc, (c | k) ? 1u : 0u);
-          }
-        }
+        constexpr uint64_t ac = C::CHUNK_BYTES >> 4, bc = C::Q_CHUNK >> 4;
+        umma_ss<0>(d, ad, bd, idesc);
+        umma_ss<1>(d, ad + 2, bd + 2, idesc);
+        umma_ss<1>(d, ad + 4, bd + 4, idesc);
+        umma_ss<1>(d, ad + 6, bd + 6, idesc);
+        umma_ss<1>(d, ad + ac, bd + bc, idesc);
+        umma_ss<1>(d, ad + ac + 2, bd + bc + 2, idesc);
+        umma_ss<1>(d, ad + ac + 4, bd + bc + 4, idesc);
+        umma_ss<1>(d, ad + ac + 6, bd + bc + 6, idesc);
         mma_commit(&op_empty[s]);
         mma_commit(&acc_full[a]);
         ++i;

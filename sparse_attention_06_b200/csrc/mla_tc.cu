@@ -6,17 +6,23 @@
 // where V is the first 512 dims of the same rows.  The softmax is the usual scaled one.
 //
 // Work unit = (query t, key split sp, value half v).  A unit computes, for its slice of the
-// query's selected rows (32-row tiles), S = Q K^T on the tensor cores (M = 128 heads, N = 32 rows,
+// query's selected rows (64-row tiles), S = Q K^T on the tensor cores (M = 128 heads, N = 64 rows,
 // K = 576), an online softmax per head row, and O_v += P V_v (M = 128 heads, N = 256 value dims,
-// K = 32 rows) into tensor memory.  Tensor memory holds O_v (256 columns) and two S buffers
-// (32 columns each): the full O (512 columns) would leave no room for S, so the two value halves
-// run on two CTAs, each recomputing S.  Q (128 x 576 bf16, 144 KB) stays in shared memory for the
-// whole unit; rows are gathered from the paged pool with cp.async into a two-stage ring.
+// K = 64 rows) into tensor memory.  The full O (512 f32 columns) would fill tensor memory, so the
+// two value halves run on two CTAs, each recomputing S.
+// Tensor memory (512 columns): O_v [0, 256), S [256, 320), and the first 384 dims of Q
+// [320, 512) -- the S products read those as the A operand straight from tensor memory, so only
+// Q's last 192 dims (48 KB) are read from shared memory.  Shared memory holds a two-stage ring of
+// gathered rows (72 KB per 64-row tile, 128B-swizzled: the same bytes serve as the K-major B of
+// Q K^T and the MN-major B of P V) and P (16 KB).  A tensor-core instruction costs a roughly fixed
+// issue time of ~40-50 cycles below N = 128, so 64-row tiles halve the issue cost per row
+// against 32-row tiles.
 // With several key splits per query each unit writes (O / l, LSE) partials that a small combine
 // kernel merges: O = sum_sp exp(LSE_sp - LSE) O_sp, LSE = log sum_sp exp(LSE_sp).
 //
-// Roles (224 threads): warps 0-1 gather rows (warp 0 lane 0 also loads Q by TMA), warp 2 owns
-// TMEM and issues the MMAs, warps 3-6 run the softmax and the epilogue (one head row per thread).
+// Roles (288 threads): warps 0-3 gather rows with cp.async and write Q into tensor memory (warp
+// 0 lane 0 also loads Q's shared-memory part by TMA), warp 4 owns tensor memory and issues the
+// MMAs, warps 5-8 run the softmax and the epilogue (one head row per thread).
 // All waits are bounded; bad indices / block ids set the device error word and are skipped.
 #include <cuda.h>
 #include <math.h>
@@ -32,33 +38,39 @@ constexpr int kH = 128;         // heads (MMA M)
 constexpr int kDqk = 576;       // latent + rope
 constexpr int kDv = 512;        // value dims
 constexpr int kHalf = 256;      // value dims per CTA
-constexpr int kTile = 32;       // rows per tile (MMA N of Q K^T, MMA K of P V)
+constexpr int kTile = 64;       // rows per tile (MMA N of Q K^T, MMA K of P V)
 constexpr int kChunks = 9;      // 64-dim column blocks of a row
+constexpr int kTmemQChunks = 6; // Q column blocks held in tensor memory
 constexpr int kPage = 64;
-constexpr int kThreads = 224;
+constexpr int kStages = 2;      // gathered-row ring
+constexpr int kGatherWarps = 4;
+constexpr int kKeysPerWarp = kTile / kGatherWarps;  // 16
+constexpr int kThreads = 32 * (kGatherWarps + 1 + 4);
 
-constexpr int Q_CHUNK = kH * 128;            // 16 KB: 128 head rows x 64 dims
-constexpr int Q_BYTES = kChunks * Q_CHUNK;   // 144 KB
-constexpr int K_CHUNK = kTile * 128;         // 4 KB: 32 rows x 64 dims
-constexpr int K_BYTES = kChunks * K_CHUNK;   // 36 KB
-constexpr int P_BYTES = kH * kTile * 2;      // 8 KB
+constexpr int Q_CHUNK = kH * 128;                            // 16 KB: 128 head rows x 64 dims
+constexpr int QS_BYTES = (kChunks - kTmemQChunks) * Q_CHUNK; // 48 KB of Q in shared memory
+constexpr int K_CHUNK = kTile * 128;                         // 8 KB: 64 rows x 64 dims
+constexpr int K_BYTES = kChunks * K_CHUNK;                   // 72 KB
+constexpr int P_BYTES = kH * kTile * 2;                      // 16 KB
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + Q_BYTES;
-constexpr int OFF_P = OFF_K + 2 * K_BYTES;
+constexpr int OFF_K = OFF_Q + QS_BYTES;
+constexpr int OFF_P = OFF_K + kStages * K_BYTES;
 constexpr int OFF_BAR = OFF_P + P_BYTES;
-constexpr int NBAR = 15;
-constexpr int OFF_MASK = OFF_BAR + NBAR * 8;   // valid-row masks: 2 stages x 2 gather warps
-constexpr int OFF_MISC = OFF_MASK + 16;
+constexpr int NBAR = 2 + 3 * kStages + 5;
+constexpr int OFF_MASK = OFF_BAR + NBAR * 8;                 // valid-row masks [stage][gather warp]
+constexpr int OFF_MISC = OFF_MASK + kStages * kGatherWarps * 4;
 constexpr int BYTES = OFF_MISC + 32;
 constexpr int SMEM = BYTES + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
 
 constexpr uint32_t TM_O = 0;       // O half: columns [0, 256)
-constexpr uint32_t TM_S = 256;     // S buffers: [256, 288), [288, 320)
+constexpr uint32_t TM_S = 256;     // S: [256, 320)
+constexpr uint32_t TM_Q = 320;     // Q dims [0, 384) as bf16 pairs: [320, 512)
 constexpr uint32_t TM_COLS = 512;
 
 struct Params {
   const __nv_bfloat16* latent;   // pool rows of 576
+  const __nv_bfloat16* q;        // [T, 128, 576]
   const int32_t* idx;
   const int32_t* q_req;
   const int32_t* q_pos;
@@ -87,7 +99,8 @@ __device__ __forceinline__ void unit_coords(const Params& p, int u, int& t, int&
 }
 
 // Row lookup of selection slot `slot` of query t in two halves, so that the dependent loads
-// can be issued a tile apart: the selected position of a slot (kNoSlot when the slot is outside the split or the selection) ...
+// can be issued a tile apart: the selected position of a slot (kNoSlot when the slot is outside
+// the split or the selection) ...
 constexpr int kNoSlot = -2;
 __device__ __forceinline__ int slot_pos(const Params& p, int t, bool qok, int sp, int slot) {
   if (!qok || slot >= min(p.k, (sp + 1) * p.ks)) return kNoSlot;
@@ -123,16 +136,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* k_ring = smem + OFF_K;
   uint8_t* p_s = smem + OFF_P;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* q_full = bars + 0;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;   // [2]
-  uint64_t* k_empty = bars + 4;  // [2]
-  uint64_t* s_full = bars + 6;   // [2]
-  uint64_t* s_empty = bars + 8;  // [2]
-  uint64_t* p_full = bars + 10;
-  uint64_t* pv_done = bars + 11;
-  uint64_t* mma_fin = bars + 12;
-  uint64_t* m_full = bars + 13;  // [2] valid-row mask of a stage published
+  uint64_t* q_full = bars + 0;                 // Q of the unit in place (TMEM part + smem part)
+  uint64_t* q_empty = bars + 1;                // the unit's last Q K^T has completed
+  uint64_t* k_full = bars + 2;                 // [kStages] rows landed
+  uint64_t* k_empty = k_full + kStages;        // [kStages] P V of the stage done
+  uint64_t* m_full = k_empty + kStages;        // [kStages] valid-row masks published
+  uint64_t* s_full = m_full + kStages;         // S computed
+  uint64_t* s_empty = s_full + 1;              // S read by the softmax
+  uint64_t* p_full = s_empty + 1;              // P written
+  uint64_t* pv_done = p_full + 1;              // P V completed
+  uint64_t* mma_fin = pv_done + 1;
   uint32_t* masks = reinterpret_cast<uint32_t*>(smem + OFF_MASK);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 8);
@@ -141,23 +154,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int units = p.T * p.nsplit * 2;
 
   if (tid == 0) {
-    mbar_init(q_full, 1);
+    mbar_init(q_full, 32 * kGatherWarps + 1);
     mbar_init(q_empty, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&k_full[i], 64);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&k_full[i], 32 * kGatherWarps);
       mbar_init(&k_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
+      mbar_init(&m_full[i], kGatherWarps);
     }
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, 4);
     mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
     mbar_init(mma_fin, 1);
-    mbar_init(&m_full[0], 2);
-    mbar_init(&m_full[1], 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 2) {
+  if (warp == kGatherWarps) {
     tmem_alloc(tmem_slot, TM_COLS);
     tmem_relinquish();
   }
@@ -166,81 +178,100 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < 2) {
-    // ------------------------------------------------------------------ Q TMA + row gather
-    const int gw = warp;  // rows 16*gw .. 16*gw+15 of each tile
-    int gi = 0;           // CTA-wide tile counter
-    int ui = 0;           // CTA-wide unit counter
+  if (warp < kGatherWarps) {
+    // ------------------------------------------------------------------ Q and row gather
+    const int gw = warp;                  // keys gw*16 .. gw*16+15 of each tile; head rows gw*32..
+    const int h = gw * 32 + lane;
+    const uint32_t my_lanes = tmem + ((uint32_t)(gw * 32) << 16);
+    int gi = 0;  // CTA-wide tile counter
+    int ui = 0;  // CTA-wide unit counter
     bool ok = true;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
       int t, sp, v;
       unit_coords(p, u, t, sp, v);
+      // Q: the previous unit's Q K^T products must be done with it
+      if (ui >= 1 && !(ok = warp_wait(q_empty, (ui - 1) & 1, p.err, abort_flag))) break;
+      tc_fence_after();
+      if (gw == 0 && lane == 0) {
+        mbar_arrive_expect_tx(q_full, QS_BYTES);
+        for (int c = kTmemQChunks; c < kChunks; ++c)
+          tma_load_2d(q_s + (c - kTmemQChunks) * Q_CHUNK, &qmap, q_full, c * 64, t * kH);
+      }
+      {
+        // this thread's head row, dims 0..383, into tensor-memory columns [320, 512)
+        const uint4* src = reinterpret_cast<const uint4*>(p.q + ((int64_t)t * kH + h) * kDqk);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {  // 96 dims = 48 columns per batch
+          uint32_t w[48];
+#pragma unroll
+          for (int e = 0; e < 12; ++e) {
+            const uint4 x = __ldg(src + b * 12 + e);
+            w[4 * e] = x.x; w[4 * e + 1] = x.y; w[4 * e + 2] = x.z; w[4 * e + 3] = x.w;
+          }
+          tmem_st16(my_lanes + TM_Q + b * 48, *reinterpret_cast<uint32_t(*)[16]>(&w[0]));
+          tmem_st16(my_lanes + TM_Q + b * 48 + 16, *reinterpret_cast<uint32_t(*)[16]>(&w[16]));
+          tmem_st16(my_lanes + TM_Q + b * 48 + 32, *reinterpret_cast<uint32_t(*)[16]>(&w[32]));
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(q_full);
+      }
       const int req = p.q_req[t];
       const int pos = p.q_pos[t];
       const bool qok = req >= 0 && req < p.num_reqs && pos >= 0 && pos < p.max_context;
       if (!qok && tid == 0 && v == 0 && sp == 0) raise_error(p.err, DSA_DEVERR_REQUEST);
-      if (warp == 0) {
-        if (ui >= 1 && !(ok = warp_wait(q_empty, (ui - 1) & 1, p.err, abort_flag))) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(q_full, Q_BYTES);
-          for (int c = 0; c < kChunks; ++c) tma_load_2d(q_s + c * Q_CHUNK, &qmap, q_full, c * 64, t * kH);
-        }
-      }
       const int ntiles = unit_tiles(p, sp);
       // Row lookups of this warp's 16 keys per tile (lanes 0..15), software-pipelined so that no
       // load is waited on in the tile it is issued: the selected position two tiles ahead and the
       // block id one tile ahead.
-      const bool mine = lane < 16;
-      const int kslot = sp * p.ks + gw * 16 + lane;
+      const bool mine = lane < kKeysPerWarp;
+      const int kslot = sp * p.ks + gw * kKeysPerWarp + lane;
       int ps_j = mine && ntiles > 0 ? slot_pos(p, t, qok, sp, kslot) : kNoSlot;
       int ps_j1 = mine && ntiles > 1 ? slot_pos(p, t, qok, sp, kslot + kTile) : kNoSlot;
       int blk_j = mine ? pos_block(p, req, pos, ps_j, v == 0) : -1;
       for (int j = 0; j < ntiles; ++j, ++gi) {
-        const int s = gi & 1;
+        const int s = gi % kStages;
         const int64_t row = blk_j >= 0 ? (int64_t)blk_j * kPage + (ps_j % kPage) : -1;
         const int blk_j1 = mine && j + 1 < ntiles ? pos_block(p, req, pos, ps_j1, v == 0) : -1;
         const int ps_j2 = mine && j + 2 < ntiles ? slot_pos(p, t, qok, sp, kslot + (j + 2) * kTile) : kNoSlot;
-        if (gi >= 2 && !(ok = warp_wait(&k_empty[s], ((gi >> 1) - 1) & 1, p.err, abort_flag))) break;
-        // publish which rows of the tile are real to the softmax warps
-        const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, row >= 0) & 0xFFFFu;
+        if (gi >= kStages && !(ok = warp_wait(&k_empty[s], ((gi / kStages) - 1) & 1, p.err, abort_flag))) break;
+        // publish which of this warp's rows are real to the softmax warps
+        const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, row >= 0) & ((1u << kKeysPerWarp) - 1u);
         if (lane == 0) {
-          masks[s * 2 + gw] = vmask;
+          masks[s * kGatherWarps + gw] = vmask;
           mbar_arrive(&m_full[s]);
         }
         ps_j = ps_j1;
         ps_j1 = ps_j2;
         blk_j = blk_j1;
-        uint8_t* stage = k_ring + s * K_BYTES;
-        const uint32_t stage_u32 = smem_u32(stage);
-#pragma unroll 1
-        for (int kk = 0; kk < 16; ++kk) {
-          const int64_t r = __shfl_sync(0xFFFFFFFFu, row, kk);
-          const int key = gw * 16 + kk;
-          const char* src = reinterpret_cast<const char*>(p.latent) + (r >= 0 ? r : 0) * (kDqk * 2);
-          const uint32_t nbytes = r >= 0 ? 16u : 0u;
-#pragma unroll
-          for (int rep = 0; rep < 3; ++rep) {
-            const int piece = lane + 32 * rep;  // 72 pieces of 16 bytes per row
-            if (piece < 72) {
-              const int c = piece >> 3, sub = piece & 7;
-              cp_async_16(stage_u32 + c * K_CHUNK + sw128_offset(key, sub), src + piece * 16, nbytes);
-            }
-          }
+        const uint32_t stage_u32 = smem_u32(k_ring + s * K_BYTES);
+        // 16 rows x 72 pieces of 16 bytes = 36 per lane; 32 consecutive pieces per step
+#pragma unroll 4
+        for (int r = 0; r < 36; ++r) {
+          const int piece = lane + 32 * r;
+          const int kk = piece / 72, q16 = piece % 72;
+          const int64_t rw = __shfl_sync(0xFFFFFFFFu, row, kk);
+          const int key = gw * kKeysPerWarp + kk;
+          const char* src = reinterpret_cast<const char*>(p.latent) + (rw >= 0 ? rw : 0) * (kDqk * 2) + q16 * 16;
+          cp_async_16(stage_u32 + (q16 >> 3) * K_CHUNK + sw128_offset(key, q16 & 7), src, rw >= 0 ? 16u : 0u);
         }
         cp_async_mbar_arrive_noinc(&k_full[s]);
       }
     }
     // let every copy this thread issued land before the CTA may exit
-    cp_async_wait<0>();
-  } else if (warp == 2) {
+    cp_async_wait_all();
+  } else if (warp == kGatherWarps) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = idesc_f16(1u, 0u, 128u, (uint32_t)kTile);  // S: B K-major
       const uint32_t idesc_o = idesc_f16(1u, 1u, 128u, (uint32_t)kHalf);  // O: B (V) MN-major
       int gi = 0, ui = 0;
       bool ok = true;
-      const uint32_t q_base = smem_u32(q_s);
-      const uint32_t p_base = smem_u32(p_s);
+      const uint64_t qd = sw128_desc(smem_u32(q_s), 16, 1024);
+      // P [128 x 64] K-major, no swizzle: 8x16-byte core matrices 128 B apart along K and 1024 B
+      // apart along M; one K step (16 keys) is two core matrices = 256 bytes
+      const uint64_t pd = noswz_desc(smem_u32(p_s), 128, 1024);
+      const uint32_t d_s = tmem + TM_S, d_o = tmem + TM_O, a_q = tmem + TM_Q;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
         int t, sp, v;
         unit_coords(p, u, t, sp, v);
@@ -249,41 +280,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ntiles == 0) mma_commit(q_empty);
         for (int j = 0; j <= ntiles && ok; ++j) {
           if (j < ntiles) {
-            // S[gi] = Q K^T
-            const int g = gi + j, s = g & 1;
-            if (!(ok = mbar_wait(&k_full[s], (g >> 1) & 1, p.err, abort_flag))) break;
-            if (g >= 2 && !(ok = mbar_wait(&s_empty[s], ((g >> 1) - 1) & 1, p.err, abort_flag))) break;
+            // S[gi + j] = Q K^T: Q dims 0..383 from tensor memory, 384..575 from shared memory
+            const int g = gi + j, s = g % kStages;
+            if (!(ok = mbar_wait(&k_full[s], (g / kStages) & 1, p.err, abort_flag))) break;
+            if (g >= 1 && !(ok = mbar_wait(s_empty, (g - 1) & 1, p.err, abort_flag))) break;
             fence_proxy_async_smem();
             tc_fence_after();
-            const uint32_t k_base = smem_u32(k_ring + s * K_BYTES);
-            const uint32_t d = tmem + TM_S + (uint32_t)(s * kTile);
-#pragma unroll 1
-            for (int c = 0; c < kChunks; ++c) {
+            const uint64_t kd = sw128_desc(smem_u32(k_ring + s * K_BYTES), 16, 1024);
+            constexpr uint64_t kc = K_CHUNK >> 4, qc = Q_CHUNK >> 4;
+            umma_ts<0>(d_s, a_q + 0, kd + 0, idesc_s);
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = sw128_desc(q_base + c * Q_CHUNK + kk * 32, 16, 1024);
-                const uint64_t bd = sw128_desc(k_base + c * K_CHUNK + kk * 32, 16, 1024);
-                mma_f16_ss(d, ad, bd, idesc_s, (c | kk) ? 1u : 0u);
-              }
-            }
-            mma_commit(&s_full[s]);
+            for (int i = 1; i < 4 * kTmemQChunks; ++i)  // chunk i/4, K step i%4: 8 TMEM columns, 32 B
+              umma_ts<1>(d_s, a_q + (uint32_t)(i * 8), kd + (uint64_t)(i >> 2) * kc + (uint64_t)(i & 3) * 2, idesc_s);
+#pragma unroll
+            for (int i = 0; i < 4 * (kChunks - kTmemQChunks); ++i)
+              umma_ss<1>(d_s, qd + (uint64_t)(i >> 2) * qc + (uint64_t)(i & 3) * 2,
+                         kd + (uint64_t)(kTmemQChunks + (i >> 2)) * kc + (uint64_t)(i & 3) * 2, idesc_s);
+            mma_commit(s_full);
             if (j == ntiles - 1) mma_commit(q_empty);  // last use of Q by this unit
           }
           if (j >= 1) {
-            // O_v += P[gi + j - 1] V_v
-            const int g = gi + j - 1, s = g & 1;
+            // O_v += P[gi + j - 1] V_v; V is MN-major 128B-swizzled: 64-dim blocks K_CHUNK apart,
+            // 8-row groups 1024 B apart, one K step (16 rows) = 2048 bytes
+            const int g = gi + j - 1, s = g % kStages;
             if (!(ok = mbar_wait(p_full, g & 1, p.err, abort_flag))) break;
             tc_fence_after();
-            const uint32_t v_base = smem_u32(k_ring + s * K_BYTES) + (uint32_t)(v * 4 * K_CHUNK);
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-              // A = P [128 x 32] K-major, no swizzle: 8x16B core matrices, 128 B apart along K,
-              // 512 B apart along M.  B = V [256 x 32] MN-major 128B-swizzled: 64-dim blocks
-              // K_CHUNK apart, 8-row groups 1024 B apart.
-              const uint64_t ad = noswz_desc(p_base + kk * 256, 128, 512);
-              const uint64_t bd = sw128_desc(v_base + kk * 2048, K_CHUNK, 1024);
-              mma_f16_ss(tmem + TM_O, ad, bd, idesc_o, (j > 1 || kk) ? 1u : 0u);
-            }
+            const uint64_t vd = sw128_desc(smem_u32(k_ring + s * K_BYTES) + (uint32_t)(v * 4 * K_CHUNK), K_CHUNK, 1024);
+            if (j > 1)
+              umma_ss<1>(d_o, pd, vd, idesc_o);
+            else
+              umma_ss<0>(d_o, pd, vd, idesc_o);
+            umma_ss<1>(d_o, pd + 16, vd + 128, idesc_o);
+            umma_ss<1>(d_o, pd + 32, vd + 256, idesc_o);
+            umma_ss<1>(d_o, pd + 48, vd + 384, idesc_o);
             mma_commit(pv_done);
             mma_commit(&k_empty[s]);
           }
@@ -307,24 +336,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ntiles = unit_tiles(p, sp);
       float m_used = -INFINITY, l = 0.0f;
       for (int j = 0; j < ntiles; ++j) {
-        const int g = gi + j, s = g & 1;
-        if (!(ok = warp_wait(&s_full[s], (g >> 1) & 1, p.err, abort_flag))) break;
-        if (!(ok = warp_wait(&m_full[s], (g >> 1) & 1, p.err, abort_flag))) break;
+        const int g = gi + j, s = g % kStages;
+        if (!(ok = warp_wait(s_full, g & 1, p.err, abort_flag))) break;
+        if (!(ok = warp_wait(&m_full[s], (g / kStages) & 1, p.err, abort_flag))) break;
         tc_fence_after();
-        uint32_t sv[32];
-        tmem_ld16(lane_base + TM_S + s * kTile, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-        tmem_ld16(lane_base + TM_S + s * kTile + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+        uint32_t sv[64];
+        tmem_ld16(lane_base + TM_S, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+        tmem_ld16(lane_base + TM_S + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+        tmem_ld16(lane_base + TM_S + 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[32]));
+        tmem_ld16(lane_base + TM_S + 48, *reinterpret_cast<uint32_t(*)[16]>(&sv[48]));
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[s]);
-        const uint32_t valid = masks[s * 2 + 0] | (masks[s * 2 + 1] << 16);
-        float x[32];
+        if (lane == 0) mbar_arrive(s_empty);
+        uint64_t valid = 0u;
+#pragma unroll
+        for (int w = 0; w < kGatherWarps; ++w) valid |= (uint64_t)masks[s * kGatherWarps + w] << (w * kKeysPerWarp);
         float mt = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] = ((valid >> c) & 1u) ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
-          mt = fmaxf(mt, x[c]);
+        for (int c = 0; c < 64; ++c) {
+          const float xv = ((valid >> c) & 1u) ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
+          sv[c] = __float_as_uint(xv);
+          mt = fmaxf(mt, xv);
         }
         // the P buffer and O are free once the previous tile's P V has completed
         if (g >= 1 && !(ok = warp_wait(pv_done, (g - 1) & 1, p.err, abort_flag))) break;
@@ -339,13 +372,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             // rescale this row of O before the next P V accumulates into it
             tc_fence_after();
 #pragma unroll 1
-            for (int c0 = 0; c0 < kHalf; c0 += 16) {
-              uint32_t o[16];
-              tmem_ld16(lane_base + TM_O + c0, o);
+            for (int c0 = 0; c0 < kHalf; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld16(lane_base + TM_O + c0, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+              tmem_ld16(lane_base + TM_O + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
               tmem_wait_ld();
 #pragma unroll
-              for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
-              tmem_st16(lane_base + TM_O + c0, o);
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+              tmem_st16(lane_base + TM_O + c0, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+              tmem_st16(lane_base + TM_O + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
             }
             tmem_wait_st();
           }
@@ -353,11 +388,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = m_new;
         }
         float psum = 0.0f;
-        uint32_t pk[16];
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float p0 = x[c] == -INFINITY ? 0.0f : exp2f(x[c] - m_used);
-          const float p1 = x[c + 1] == -INFINITY ? 0.0f : exp2f(x[c + 1] - m_used);
+        for (int c = 0; c < 64; c += 2) {
+          const float x0 = __uint_as_float(sv[c]), x1 = __uint_as_float(sv[c + 1]);
+          const float p0 = x0 == -INFINITY ? 0.0f : exp2f(x0 - m_used);
+          const float p1 = x1 == -INFINITY ? 0.0f : exp2f(x1 - m_used);
           const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
           // the normaliser sums the rounded weights that P V actually uses
           const float2 bf = __bfloat1622float2(b);
@@ -365,10 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&b);
         }
         l += psum;
-        // P row r: 4 core-matrix rows of 16 B (8 keys each), no swizzle
-        uint8_t* prow = p_s + (r >> 3) * 512 + (r & 7) * 16;
+        // P row r: 8 core-matrix rows of 16 B (8 keys each), no swizzle
+        uint8_t* prow = p_s + (r >> 3) * 1024 + (r & 7) * 16;
 #pragma unroll
-        for (int kc = 0; kc < 4; ++kc)
+        for (int kc = 0; kc < 8; ++kc)
           *reinterpret_cast<uint4*>(prow + kc * 128) = make_uint4(pk[4 * kc], pk[4 * kc + 1], pk[4 * kc + 2], pk[4 * kc + 3]);
         fence_proxy_async_smem();
         tc_fence_before();
@@ -430,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == kGatherWarps) {
     tc_fence_after();
     tmem_dealloc(tmem, TM_COLS);
   }
@@ -492,7 +528,7 @@ int splits_for(int T, int k, int num_sms) {
   int best = 1;
   for (int n = 1; n <= kMaxSplits; n *= 2) {
     int ks = ((k + n - 1) / n + kTile - 1) / kTile * kTile;
-    if (ks < 2 * kTile && n > 1) break;
+    if (ks < kTile) break;
     const int ns = (k + ks - 1) / ks;
     const long long units = 2LL * T * ns;
     const double per_cta = (double)((units + num_sms - 1) / num_sms) * (ks / kTile);
@@ -521,6 +557,7 @@ cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_
   if (!encode_tmap_2d(&qmap, a.q, 2, kDqk, (uint64_t)T * kH, kDqk * 2, 64, kH, true)) return cudaErrorInvalidValue;
   Params p;
   p.latent = static_cast<const __nv_bfloat16*>(a.latent.data);
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.idx = a.idx;
   p.q_req = a.batch.q_req;
   p.q_pos = a.batch.q_pos;
