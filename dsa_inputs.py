@@ -237,6 +237,17 @@ def profile_decode(B=8, L=65536, seed=0x5EED + 5) -> Spec:
                 q_pos=[L - 1] * B, seed=seed)
 
 
+def profile_prefill(ctx=16384, chunk=1024, seed=0x5EED + 6) -> Spec:
+    """A smaller prefill chunk (e4m3 keys) for profiling captures."""
+    return prefill(ctx=ctx, chunk=chunk, seed=seed)
+
+
+def profile_long(B=8, L=202752, seed=0x5EED + 7) -> Spec:
+    """Long-context e4m3 decode at batch 8 (about 2 GB resident) for profiling captures."""
+    return Spec("profile_long_e4m3_B%d_L%d" % (B, L), lens=[L] * B, q_req=list(range(B)),
+                q_pos=[L - 1] * B, key_dtype="e4m3", seed=seed)
+
+
 WORKLOADS = {
     "tiny": tiny,
     "decode": decode,
@@ -244,6 +255,8 @@ WORKLOADS = {
     "prefill": prefill,
     "long_decode": long_decode,
     "profile_decode": profile_decode,
+    "profile_prefill": profile_prefill,
+    "profile_long": profile_long,
 }
 
 

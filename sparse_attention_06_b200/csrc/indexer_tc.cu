@@ -6,9 +6,10 @@
 // with 64 indexer heads of 128 dims, bf16 queries, and bf16 keys or e4m3 keys with a per-token
 // scale (khat = code * scale; for scale > 0 the scale is applied after the head sum, which is the
 // same value).  bf16 keys multiply bf16 queries exactly as stored.  For e4m3 keys the product runs
-// in f16: every e4m3 code is exact in f16 (one conversion instruction per pair), and each query
-// tile is converted bf16 -> f16 once, which is exact for |q| in [2^-14, 65504] (smaller values
-// keep an absolute error below 2^-25).
+// in f16: each code is re-encoded by integer bit operations as the f16 holding code * 2^-8 (exact
+// for every finite code, subnormals included), the epilogue multiplies the per-token scale by 2^8,
+// and each query tile is converted bf16 -> f16 once, which is exact for |q| in [2^-14, 65504]
+// (smaller values keep an absolute error below 2^-25).
 //
 // Shape of the computation: per tile of 128 consecutive key positions (two 64-token pages of the
 // paged key cache) one tensor-core product D[128 keys, 64*NQ] = K[128 keys, 128] . Q[64*NQ, 128]^T
@@ -172,21 +173,25 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* 
   mbar_wait(bar, parity, err, nullptr);
 }
 
-// fp8 e4m3 x16 -> f16 x16 (exact: every e4m3 value is an f16 value)
+// Two e4m3 codes -> two f16 holding code * 2^-8, exactly.  An e4m3 code s.eeee.mmm has value
+// (1 + m/8) 2^(e-7) (or (m/8) 2^-6 when e = 0); its 7 magnitude bits placed at f16 bits 7..13 read
+// as (1 + m/8) 2^(e-15) (or, as an f16 subnormal, (m/8) 2^-14): the same value times 2^-8 in both
+// cases.  The sign moves from bit 7 to bit 15.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_times_2m8(uint32_t w, uint32_t byte_sel) {
+  const uint32_t x = __byte_perm(w, 0u, byte_sel);  // code a in bits 0..7, code b in bits 16..23
+  return ((x << 7) & 0x3F803F80u) | ((x << 8) & 0x80008000u);
+}
+
+// fp8 e4m3 x16 -> f16 x16, each value scaled by 2^-8 (exact)
 __device__ __forceinline__ void e4m3x16_to_f16(const uint4& in, uint4& lo, uint4& hi) {
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(&in);
-  uint32_t outw[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-#pragma unroll
-    for (int hpart = 0; hpart < 2; ++hpart) {
-      const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * hpart)) & 0xFFFFu);
-      const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-      outw[2 * i + hpart] = (uint32_t)h2.x | ((uint32_t)h2.y << 16);
-    }
-  }
-  lo = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-  hi = make_uint4(outw[4], outw[5], outw[6], outw[7]);
+  lo.x = e4m3x2_to_f16x2_times_2m8(in.x, 0x4140u);
+  lo.y = e4m3x2_to_f16x2_times_2m8(in.x, 0x4342u);
+  lo.z = e4m3x2_to_f16x2_times_2m8(in.y, 0x4140u);
+  lo.w = e4m3x2_to_f16x2_times_2m8(in.y, 0x4342u);
+  hi.x = e4m3x2_to_f16x2_times_2m8(in.z, 0x4140u);
+  hi.y = e4m3x2_to_f16x2_times_2m8(in.z, 0x4342u);
+  hi.z = e4m3x2_to_f16x2_times_2m8(in.w, 0x4140u);
+  hi.w = e4m3x2_to_f16x2_times_2m8(in.w, 0x4342u);
 }
 
 // bf16 x8 -> f16 x8 in place (16 bytes)
@@ -400,7 +405,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
       } else {
         g2 = -1;
       }
-      if (FP8 && b1 >= 0) sc1 = p.key_scale[(int64_t)b1 * kPage + (r & 63)];
+      if (FP8 && b1 >= 0) sc1 = 256.0f * p.key_scale[(int64_t)b1 * kPage + (r & 63)];
     } else {
       g1 = -1;
     }
@@ -412,7 +417,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
       g0 = g1; j0 = j1; G0 = G1; b0 = b1; sc0 = sc1;
       g1 = g2; j1 = j2; G1 = G2; b1 = b2;
       sc1 = 1.0f;
-      if (g1 >= 0 && FP8 && b1 >= 0) sc1 = p.key_scale[(int64_t)b1 * kPage + (r & 63)];
+      if (g1 >= 0 && FP8 && b1 >= 0) sc1 = 256.0f * p.key_scale[(int64_t)b1 * kPage + (r & 63)];  // undo 2^-8
       if (g1 >= 0 && W.next(p, g2, j2)) {
         G2 = W.G;
         b2 = page_block(p, G2, j2, pg, false);

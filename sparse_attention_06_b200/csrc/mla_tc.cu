@@ -85,6 +85,14 @@ struct Params {
   int* err;
 };
 
+// 2^x by the hardware approximation (relative error ~2^-22, far below the bf16 rounding of P);
+// 2^-inf = 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -278,43 +286,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ntiles = unit_tiles(p, sp);
         if (!(ok = mbar_wait(q_full, ui & 1, p.err, abort_flag))) break;
         if (ntiles == 0) mma_commit(q_empty);
-        for (int j = 0; j <= ntiles && ok; ++j) {
-          if (j < ntiles) {
-            // S[gi + j] = Q K^T: Q dims 0..383 from tensor memory, 384..575 from shared memory
-            const int g = gi + j, s = g % kStages;
-            if (!(ok = mbar_wait(&k_full[s], (g / kStages) & 1, p.err, abort_flag))) break;
-            if (g >= 1 && !(ok = mbar_wait(s_empty, (g - 1) & 1, p.err, abort_flag))) break;
-            fence_proxy_async_smem();
-            tc_fence_after();
-            const uint64_t kd = sw128_desc(smem_u32(k_ring + s * K_BYTES), 16, 1024);
-            constexpr uint64_t kc = K_CHUNK >> 4, qc = Q_CHUNK >> 4;
-            umma_ts<0>(d_s, a_q + 0, kd + 0, idesc_s);
-#pragma unroll
-            for (int i = 1; i < 4 * kTmemQChunks; ++i)  // chunk i/4, K step i%4: 8 TMEM columns, 32 B
-              umma_ts<1>(d_s, a_q + (uint32_t)(i * 8), kd + (uint64_t)(i >> 2) * kc + (uint64_t)(i & 3) * 2, idesc_s);
-#pragma unroll
-            for (int i = 0; i < 4 * (kChunks - kTmemQChunks); ++i)
-              umma_ss<1>(d_s, qd + (uint64_t)(i >> 2) * qc + (uint64_t)(i & 3) * 2,
-                         kd + (uint64_t)(kTmemQChunks + (i >> 2)) * kc + (uint64_t)(i & 3) * 2, idesc_s);
-            mma_commit(s_full);
-            if (j == ntiles - 1) mma_commit(q_empty);  // last use of Q by this unit
+        // Issue whichever is ready: P V of the oldest finished softmax first (it frees a ring stage
+        // and lets the softmax move on), else the next tile's Q K^T.
+        int ns = 0, np = 0;
+        long long last = clock64();
+        while (np < ntiles) {
+          bool did = false;
+          if (np < ns) {
+            const int g = gi + np, s = g % kStages;
+            if (mbar_try_wait(p_full, g & 1)) {
+              // O_v += P V_v; V is MN-major 128B-swizzled: 64-dim blocks K_CHUNK apart, 8-row
+              // groups 1024 B apart, one K step (16 rows) = 2048 bytes
+              tc_fence_after();
+              const uint64_t vd = sw128_desc(smem_u32(k_ring + s * K_BYTES) + (uint32_t)(v * 4 * K_CHUNK), K_CHUNK, 1024);
+              if (np > 0)
+                umma_ss<1>(d_o, pd, vd, idesc_o);
+              else
+                umma_ss<0>(d_o, pd, vd, idesc_o);
+              umma_ss<1>(d_o, pd + 16, vd + 128, idesc_o);
+              umma_ss<1>(d_o, pd + 32, vd + 256, idesc_o);
+              umma_ss<1>(d_o, pd + 48, vd + 384, idesc_o);
+              mma_commit(pv_done);
+              mma_commit(&k_empty[s]);
+              ++np;
+              did = true;
+            }
           }
-          if (j >= 1) {
-            // O_v += P[gi + j - 1] V_v; V is MN-major 128B-swizzled: 64-dim blocks K_CHUNK apart,
-            // 8-row groups 1024 B apart, one K step (16 rows) = 2048 bytes
-            const int g = gi + j - 1, s = g % kStages;
-            if (!(ok = mbar_wait(p_full, g & 1, p.err, abort_flag))) break;
-            tc_fence_after();
-            const uint64_t vd = sw128_desc(smem_u32(k_ring + s * K_BYTES) + (uint32_t)(v * 4 * K_CHUNK), K_CHUNK, 1024);
-            if (j > 1)
-              umma_ss<1>(d_o, pd, vd, idesc_o);
-            else
-              umma_ss<0>(d_o, pd, vd, idesc_o);
-            umma_ss<1>(d_o, pd + 16, vd + 128, idesc_o);
-            umma_ss<1>(d_o, pd + 32, vd + 256, idesc_o);
-            umma_ss<1>(d_o, pd + 48, vd + 384, idesc_o);
-            mma_commit(pv_done);
-            mma_commit(&k_empty[s]);
+          if (!did && ns < ntiles) {
+            const int g = gi + ns, s = g % kStages;
+            if (mbar_try_wait(&k_full[s], (g / kStages) & 1) && (g == 0 || mbar_try_wait(s_empty, (g - 1) & 1))) {
+              // S[g] = Q K^T: Q dims 0..383 from tensor memory, 384..575 from shared memory
+              fence_proxy_async_smem();
+              tc_fence_after();
+              const uint64_t kd = sw128_desc(smem_u32(k_ring + s * K_BYTES), 16, 1024);
+              constexpr uint64_t kc = K_CHUNK >> 4, qc = Q_CHUNK >> 4;
+              umma_ts<0>(d_s, a_q + 0, kd + 0, idesc_s);
+#pragma unroll
+              for (int i = 1; i < 4 * kTmemQChunks; ++i)  // chunk i/4, K step i%4: 8 TMEM columns, 32 B
+                umma_ts<1>(d_s, a_q + (uint32_t)(i * 8), kd + (uint64_t)(i >> 2) * kc + (uint64_t)(i & 3) * 2, idesc_s);
+#pragma unroll
+              for (int i = 0; i < 4 * (kChunks - kTmemQChunks); ++i)
+                umma_ss<1>(d_s, qd + (uint64_t)(i >> 2) * qc + (uint64_t)(i & 3) * 2,
+                           kd + (uint64_t)(kTmemQChunks + (i >> 2)) * kc + (uint64_t)(i & 3) * 2, idesc_s);
+              mma_commit(s_full);
+              if (ns == ntiles - 1) mma_commit(q_empty);  // last use of Q by this unit
+              ++ns;
+              did = true;
+            }
+          }
+          if (did) {
+            last = clock64();
+          } else if (*abort_flag) {
+            ok = false;
+            break;
+          } else if (clock64() - last > kWaitCycles) {
+            raise_error(p.err, DSA_DEVERR_TIMEOUT);
+            *abort_flag = 1;
+            ok = false;
+            break;
           }
         }
         gi += ntiles;
@@ -389,11 +418,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float psum = 0.0f;
         uint32_t pk[32];
+        // 2^(x - m): x = -inf gives 0; while no real row has been seen m_used is -inf and every x is
+        // -inf, so the base 0 is used instead
+        const float msub = m_used == -INFINITY ? 0.0f : m_used;
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
-          const float x0 = __uint_as_float(sv[c]), x1 = __uint_as_float(sv[c + 1]);
-          const float p0 = x0 == -INFINITY ? 0.0f : exp2f(x0 - m_used);
-          const float p1 = x1 == -INFINITY ? 0.0f : exp2f(x1 - m_used);
+          const float p0 = fast_exp2(__uint_as_float(sv[c]) - msub);
+          const float p1 = fast_exp2(__uint_as_float(sv[c + 1]) - msub);
           const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
           // the normaliser sums the rounded weights that P V actually uses
           const float2 bf = __bfloat1622float2(b);
