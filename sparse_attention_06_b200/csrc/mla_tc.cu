@@ -130,6 +130,13 @@ __device__ __forceinline__ int pos_block(const Params& p, int req, int pos, int 
   return blk;
 }
 
+// Pull the 128 x 576 query block of query t into L2 ahead of its use (16 KB pieces).
+__device__ __forceinline__ void prefetch_q(const Params& p, int t) {
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(p.q + (int64_t)t * kH * kDqk);
+#pragma unroll 1
+  for (int off = 0; off < kH * kDqk * 2; off += 16384) prefetch_l2_bulk(src + off, 16384u);
+}
+
 __device__ __forceinline__ int unit_tiles(const Params& p, int sp) {
   const int first = sp * p.ks;
   const int n = min(p.ks, p.k - first);
@@ -162,6 +169,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int units = p.T * p.nsplit * 2;
 
   if (tid == 0) {
+    if (blockIdx.x < units) {
+      int t0, sp0, v0;
+      unit_coords(p, blockIdx.x, t0, sp0, v0);
+      prefetch_q(p, t0);
+    }
     mbar_init(q_full, 32 * kGatherWarps + 1);
     mbar_init(q_empty, 1);
     for (int i = 0; i < kStages; ++i) {
@@ -197,6 +209,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
       int t, sp, v;
       unit_coords(p, u, t, sp, v);
+      if (gw == 0 && lane == 0 && u + (int)gridDim.x < units) {
+        int tn, spn, vn;
+        unit_coords(p, u + gridDim.x, tn, spn, vn);
+        if (tn != t) prefetch_q(p, tn);  // the next unit's queries, while this one runs
+      }
+      // Row lookups of this warp's 16 keys per tile (lanes 0..15), software-pipelined so that no
+      // load is waited on in the tile it is issued: the selected position two tiles ahead and the
+      // block id one tile ahead.  The first ones are issued before the Q copy below.
+      const int req = p.q_req[t];
+      const int pos = p.q_pos[t];
+      const bool qok = req >= 0 && req < p.num_reqs && pos >= 0 && pos < p.max_context;
+      const int ntiles = unit_tiles(p, sp);
+      const bool mine = lane < kKeysPerWarp;
+      const int kslot = sp * p.ks + gw * kKeysPerWarp + lane;
+      int ps_j = mine && ntiles > 0 ? slot_pos(p, t, qok, sp, kslot) : kNoSlot;
+      int ps_j1 = mine && ntiles > 1 ? slot_pos(p, t, qok, sp, kslot + kTile) : kNoSlot;
       // Q: the previous unit's Q K^T products must be done with it
       if (ui >= 1 && !(ok = warp_wait(q_empty, (ui - 1) & 1, p.err, abort_flag))) break;
       tc_fence_after();
@@ -209,33 +237,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         // this thread's head row, dims 0..383, into tensor-memory columns [320, 512)
         const uint4* src = reinterpret_cast<const uint4*>(p.q + ((int64_t)t * kH + h) * kDqk);
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {  // 96 dims = 48 columns per batch
-          uint32_t w[48];
+        for (int b = 0; b < 2; ++b) {  // 192 dims = 96 columns per batch, all loads in flight
+          uint32_t w[96];
 #pragma unroll
-          for (int e = 0; e < 12; ++e) {
-            const uint4 x = __ldg(src + b * 12 + e);
+          for (int e = 0; e < 24; ++e) {
+            const uint4 x = __ldg(src + b * 24 + e);
             w[4 * e] = x.x; w[4 * e + 1] = x.y; w[4 * e + 2] = x.z; w[4 * e + 3] = x.w;
           }
-          tmem_st16(my_lanes + TM_Q + b * 48, *reinterpret_cast<uint32_t(*)[16]>(&w[0]));
-          tmem_st16(my_lanes + TM_Q + b * 48 + 16, *reinterpret_cast<uint32_t(*)[16]>(&w[16]));
-          tmem_st16(my_lanes + TM_Q + b * 48 + 32, *reinterpret_cast<uint32_t(*)[16]>(&w[32]));
+#pragma unroll
+          for (int c = 0; c < 6; ++c)
+            tmem_st16(my_lanes + TM_Q + b * 96 + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&w[c * 16]));
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(q_full);
       }
-      const int req = p.q_req[t];
-      const int pos = p.q_pos[t];
-      const bool qok = req >= 0 && req < p.num_reqs && pos >= 0 && pos < p.max_context;
       if (!qok && tid == 0 && v == 0 && sp == 0) raise_error(p.err, DSA_DEVERR_REQUEST);
-      const int ntiles = unit_tiles(p, sp);
-      // Row lookups of this warp's 16 keys per tile (lanes 0..15), software-pipelined so that no
-      // load is waited on in the tile it is issued: the selected position two tiles ahead and the
-      // block id one tile ahead.
-      const bool mine = lane < kKeysPerWarp;
-      const int kslot = sp * p.ks + gw * kKeysPerWarp + lane;
-      int ps_j = mine && ntiles > 0 ? slot_pos(p, t, qok, sp, kslot) : kNoSlot;
-      int ps_j1 = mine && ntiles > 1 ? slot_pos(p, t, qok, sp, kslot + kTile) : kNoSlot;
       int blk_j = mine ? pos_block(p, req, pos, ps_j, v == 0) : -1;
       for (int j = 0; j < ntiles; ++j, ++gi) {
         const int s = gi % kStages;
@@ -449,8 +466,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv = l > 0.0f ? 1.0f / l : 0.0f;
       const float lse = l > 0.0f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
       const int64_t orow = (int64_t)t * kH + r;
-      // O / l in 64-column pieces: four TMEM loads in flight per wait, then the stores
       const int64_t prow = ((int64_t)t * p.nsplit + sp) * kH + r;
+      // O / l leaves through this warp's 4 KB quarter of the P buffer (free: the last P V has
+      // completed), so that each global store instruction writes four whole 128-byte row pieces:
+      // lane i stages its row i (128 bytes per block, 16-byte pieces XOR-permuted by i mod 8),
+      // then the warp writes rows 4k + lane/8, piece lane mod 8.
+      uint8_t* stage = p_s + quarter * 4096;
+      const int srow = lane >> 3, spiece = lane & 7;
+      const bool f32out = p.nsplit > 1;
+      // write the staged 128-byte block of each of this warp's rows to columns [col, col + 128 B)
+      auto flush = [&](int col) {
+        __syncwarp();
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const int rr = k4 * 4 + srow;  // row within this warp's 32
+          const uint4 x = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((spiece ^ (rr & 7)) << 4));
+          if (f32out)
+            *reinterpret_cast<uint4*>(p.part_o + (prow - lane + rr) * kDv + v * kHalf + col + spiece * 4) = x;
+          else
+            *reinterpret_cast<uint4*>(p.out + (orow - lane + rr) * kDv + v * kHalf + col + spiece * 8) = x;
+        }
+        __syncwarp();
+      };
 #pragma unroll 1
       for (int c0 = 0; c0 < kHalf; c0 += 64) {
         uint32_t o[64];
@@ -464,24 +501,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 64; ++c) o[c] = 0u;
         }
-        if (p.nsplit == 1) {
-          __nv_bfloat16* dst = p.out + orow * kDv + v * kHalf + c0;
+        uint8_t* srow_ptr = stage + lane * 128;
+        if (f32out) {
+          // two blocks of 32 f32 columns
 #pragma unroll
-          for (int c = 0; c < 64; c += 8) {
-            uint32_t pk[4];
+          for (int b = 0; b < 2; ++b) {
 #pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(o[c + e]) * inv, __uint_as_float(o[c + e + 1]) * inv);
-              pk[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+            for (int j = 0; j < 8; ++j) {
+              const int c = 32 * b + 4 * j;
+              *reinterpret_cast<float4*>(srow_ptr + ((j ^ (lane & 7)) << 4)) =
+                  make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
+                              __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
             }
-            *reinterpret_cast<uint4*>(dst + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            flush(c0 + 32 * b);
           }
         } else {
-          float* dst = p.part_o + prow * kDv + v * kHalf + c0;
+          // one block of 64 bf16 columns
 #pragma unroll
-          for (int c = 0; c < 64; c += 4)
-            *reinterpret_cast<float4*>(dst + c) = make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
-                                                              __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
+          for (int j = 0; j < 8; ++j) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 hv = __floats2bfloat162_rn(__uint_as_float(o[8 * j + 2 * e]) * inv,
+                                                              __uint_as_float(o[8 * j + 2 * e + 1]) * inv);
+              pk[e] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
+            *reinterpret_cast<uint4*>(srow_ptr + ((j ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+          flush(c0);
         }
       }
       if (v == 0) {
@@ -553,23 +600,30 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const float* __restric
   if (lse_out && threadIdx.x == 0) lse_out[(int64_t)t * kH + h] = s_lse;
 }
 
+int split_size(int k, int nsplit) { return ((k + nsplit - 1) / nsplit + kTile - 1) / kTile * kTile; }
+
+// Key splits per query.  Cost model in 64-row tile times: a unit costs its tiles plus a fixed
+// ~2.5 (query load, pipeline fill, epilogue), units run in waves of one per SM, and more than one
+// split adds the combine pass (a launch, ~2 tiles, plus reading the partials, ~0.02 tile per
+// query and split).
 int splits_for(int T, int k, int num_sms) {
-  const int tiles_q = (k + kTile - 1) / kTile;  // tiles per (query, half)
-  const double ideal = 2.0 * T * tiles_q / num_sms;
+  double best_cost = 1e300;
   int best = 1;
   for (int n = 1; n <= kMaxSplits; n *= 2) {
-    int ks = ((k + n - 1) / n + kTile - 1) / kTile * kTile;
-    if (ks < kTile) break;
+    const int ks = split_size(k, n);
     const int ns = (k + ks - 1) / ks;
     const long long units = 2LL * T * ns;
-    const double per_cta = (double)((units + num_sms - 1) / num_sms) * (ks / kTile);
-    best = ns;
-    if (per_cta <= 1.1 * ideal + 1) break;
+    const double waves = (double)((units + num_sms - 1) / num_sms);
+    double cost = waves * ((double)(ks / kTile) + 2.5);
+    if (ns > 1) cost += 2.0 + 0.02 * T * ns;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = ns;
+    }
+    if (ks == kTile) break;
   }
   return best;
 }
-
-int split_size(int k, int nsplit) { return ((k + nsplit - 1) / nsplit + kTile - 1) / kTile * kTile; }
 
 }  // namespace
 

@@ -11,8 +11,9 @@
 // Fast path (rows up to 262144 positions):
 //   1. sample one 32-score chunk out of every 32 and radix-select from the sample a threshold tau
 //      expected to leave ~1.5 K scores at or above it;
-//   2. one pass over the row appends every (key, position) with key >= tau to shared memory
-//      (warp-aggregated);
+//   2. one pass over the row appends every (key, position) with key >= tau to shared memory: each
+//      warp fills its own segment with a register counter (no shared atomics), then the segments
+//      are compacted;
 //   3. if at least K and at most kCap scores were collected, the exact K-th key Tk among them is
 //      found by radix select (every score >= Tk is a candidate, so it is the row's K-th key), the
 //      keys > Tk are marked in a position bitmap, and of the keys == Tk the lowest positions are
@@ -36,14 +37,19 @@ constexpr int kMaxRow = 262144;       // bitmap capacity (positions) of the fast
 constexpr int kChunk = 32;            // sampled chunk length
 constexpr int kSampleEvery = 32;      // one chunk of every kSampleEvery
 
+constexpr int kSeg = kCap / kWarps;   // candidate segment of one warp
+constexpr int kDigitBins = 256;       // 8-bit digits of the in-shared-memory selections
+
 struct Smem {
   uint32_t hist[kBins];
   uint32_t warp_tot[kWarps + 1];
   uint32_t scal[8];
+  uint32_t red[2 * kWarps];
   uint32_t sample[kCap];    // sample keys, later the positions of the tied candidates
   uint32_t cand_key[kCap];
   uint32_t cand_pos[kCap];
   uint32_t bitmap[kMaxRow / 32];
+  uint32_t whist[kWarps * kDigitBins];  // per-warp digit histograms
 };
 
 __device__ __forceinline__ uint32_t order_key(float f, bool& is_nan) {
@@ -145,6 +151,82 @@ __device__ void radix_select(Smem& S, int64_t m, uint32_t j, Get get, uint32_t& 
   above = j - krem;
 }
 
+// Radix select over keys in shared memory (m <= kCap): the value of the j-th largest (1-based) and
+// the number of keys strictly greater.  8-bit digits counted in per-warp histograms (no atomic
+// contention between warps); digits in which every key agrees are skipped (their value is read off
+// a block-wide AND / OR of the keys).  Block-wide; every thread gets the result.
+template <class Get>
+__device__ void smem_select(Smem& S, int m, uint32_t j, Get get, uint32_t& value, uint32_t& above) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t a = 0xFFFFFFFFu, o = 0u;
+  for (int i = tid; i < m; i += kThreads) {
+    const uint32_t key = get(i);
+    a &= key;
+    o |= key;
+  }
+  for (int off = 16; off > 0; off >>= 1) {
+    a &= __shfl_xor_sync(0xFFFFFFFFu, a, off);
+    o |= __shfl_xor_sync(0xFFFFFFFFu, o, off);
+  }
+  if (lane == 0) {
+    S.red[warp] = a;
+    S.red[kWarps + warp] = o;
+  }
+  __syncthreads();
+  a = 0xFFFFFFFFu;
+  o = 0u;
+#pragma unroll 8
+  for (int w = 0; w < kWarps; ++w) {
+    a &= S.red[w];
+    o |= S.red[kWarps + w];
+  }
+  const uint32_t vary = a ^ o;          // bits that differ between keys
+  uint32_t prefix = a & ~vary;          // the agreed bits
+  uint32_t hmask = ~vary;
+  uint32_t krem = j;
+  uint32_t* wh = S.whist + warp * kDigitBins;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    const uint32_t dmask = 0xFFu << shift;
+    if ((vary & dmask) == 0u) continue;  // every key has the same digit here
+    for (int b = lane; b < kDigitBins; b += 32) wh[b] = 0u;
+    __syncwarp();
+    for (int i0 = 0; i0 < m; i0 += kThreads) {
+      const int i = i0 + tid;
+      uint32_t key = 0u;
+      bool in = false;
+      if (i < m) {
+        key = get(i);
+        in = (key & hmask) == prefix;
+      }
+      const uint32_t bin = in ? ((key >> shift) & 0xFFu) : 0xFFFFFFFFu;
+      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+      if (in && lane == __ffs(peers) - 1) atomicAdd(&wh[bin], (uint32_t)__popc(peers));  // warp-private bins
+    }
+    __syncthreads();
+    // bin totals from the top: thread t < 256 holds bin 255 - t
+    uint32_t h = 0u;
+    if (tid < kDigitBins) {
+      const int bin = kDigitBins - 1 - tid;
+#pragma unroll 8
+      for (int w = 0; w < kWarps; ++w) h += S.whist[w * kDigitBins + bin];
+    }
+    uint32_t tot;
+    const uint32_t abv = block_exclusive_scan(h, S.warp_tot, tot);
+    if (tid < kDigitBins && abv < krem && krem <= abv + h) {
+      S.scal[0] = (uint32_t)(kDigitBins - 1 - tid);
+      S.scal[1] = abv;
+    }
+    __syncthreads();
+    prefix |= S.scal[0] << shift;
+    hmask |= dmask;
+    krem -= S.scal[1];
+    __syncthreads();
+  }
+  value = prefix;
+  above = j - krem;
+}
+
 // Exact path: radix select over the row in global memory, then one in-order pass.
 __device__ void topk_exact(Smem& S, const float* row, int64_t n, int k, int32_t* out, bool& saw_nan) {
   uint32_t tk, above;
@@ -211,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t js = (int64_t)(1.5 * k * frac) + 8;
       if (js > ns) js = ns;
       uint32_t above_s;
-      radix_select(S, ns, (uint32_t)js, [&](int64_t i) { return S.sample[i]; }, tau, above_s);
+      smem_select(S, ns, (uint32_t)js, [&](int i) { return S.sample[i]; }, tau, above_s);
     }
     __syncthreads();
     // 2. collect every score at or above tau.  The row is read in 16-score groups per thread
@@ -240,6 +322,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     if (n > 0) load_group(0, cur);
+    const int warp = tid >> 5;
+    uint32_t wcount = 0u;  // candidates this warp found (warp-uniform)
     for (int64_t base = 0; base < n; base += step) {
       if (base + step < n) load_group(base + step, nxt);
 #pragma unroll
@@ -253,29 +337,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, pred);
         if (ballot) {
-          const int leader = __ffs(ballot) - 1;
-          uint32_t b0 = 0u;
-          if (lane == leader) b0 = atomicAdd(&S.scal[2], (uint32_t)__popc(ballot));
-          b0 = __shfl_sync(0xFFFFFFFFu, b0, leader);
-          if (pred) {
-            const uint32_t pos = b0 + __popc(ballot & ((1u << lane) - 1u));
-            if (pos < kCap) {
-              S.cand_key[pos] = key;
-              S.cand_pos[pos] = (uint32_t)i;
-            }
+          const uint32_t pos = wcount + __popc(ballot & ((1u << lane) - 1u));
+          if (pred && pos < (uint32_t)kSeg) {
+            S.cand_key[warp * kSeg + pos] = key;
+            S.cand_pos[warp * kSeg + pos] = (uint32_t)i;
           }
+          wcount += (uint32_t)__popc(ballot);
         }
       }
 #pragma unroll
       for (int u = 0; u < kPer; ++u) cur[u] = nxt[u];
     }
+    // compact the warp segments: read own entries, then write them at the prefix offset
+    if (lane == 0) S.red[warp] = wcount;
+    __syncthreads();
+    uint32_t off = 0u, total = 0u;
+    bool overflow = false;
+    for (int w = 0; w < kWarps; ++w) {
+      const uint32_t c = S.red[w];
+      if (w < warp) off += c;
+      total += c;
+      overflow |= c > (uint32_t)kSeg;
+    }
+    constexpr int kPerLane = kSeg / 32;
+    uint32_t mk[kPerLane], mp[kPerLane];
+#pragma unroll
+    for (int e = 0; e < kPerLane; ++e) {
+      const int idx = e * 32 + lane;
+      mk[e] = S.cand_key[warp * kSeg + idx];
+      mp[e] = S.cand_pos[warp * kSeg + idx];
+    }
+    __syncthreads();
+    if (!overflow) {
+#pragma unroll
+      for (int e = 0; e < kPerLane; ++e) {
+        const int idx = e * 32 + lane;
+        if ((uint32_t)idx < wcount) {
+          S.cand_key[off + idx] = mk[e];
+          S.cand_pos[off + idx] = mp[e];
+        }
+      }
+    }
+    if (tid == 0) S.scal[2] = overflow ? 0xFFFFFFFFu : total;
     __syncthreads();
     const uint32_t m = S.scal[2];
     fast = m >= (uint32_t)k && m <= (uint32_t)kCap;
     if (fast) {
       // 3. exact K-th key among the candidates, then mark the selection in the bitmap
       uint32_t tk, above;
-      radix_select(S, m, (uint32_t)k, [&](int64_t i) { return S.cand_key[i]; }, tk, above);
+      smem_select(S, (int)m, (uint32_t)k, [&](int i) { return S.cand_key[i]; }, tk, above);
       const uint32_t need = (uint32_t)k - above;
       const int words = (int)((n + 31) / 32);
       for (int w = tid; w < words; w += kThreads) S.bitmap[w] = 0u;
@@ -296,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (neq > need) {
         // the `need` lowest positions among the ties: radix select on the complemented position
         uint32_t v, ab;
-        radix_select(S, neq, need, [&](int64_t i) { return ~S.sample[i]; }, v, ab);
+        smem_select(S, (int)neq, need, [&](int i) { return ~S.sample[i]; }, v, ab);
         pos_cut = ~v;
       }
       for (uint32_t e = tid; e < neq; e += kThreads) {
