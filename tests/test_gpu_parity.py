@@ -112,6 +112,58 @@ def test_topk_dense_boundary_and_padding():
     check_topk(idx, s, qpos, 2048)
 
 
+def test_topk_cluster_shapes():
+    # few rows (several CTAs per row), many rows (one CTA per row), take-all rows just below and
+    # above the candidate capacity, a row stride that leaves most rows unaligned for vector loads
+    g = torch.Generator().manual_seed(9)
+    for T, ld, k in ((1, 32768, 2048), (1, 202752, 2048), (3, 9001, 2048), (40, 70000, 2048),
+                     (160, 20000, 2048), (2, 8192, 2048), (5, 40001, 100), (1, 50000, 4096)):
+        s = torch.randn(T, ld, generator=g) * 20 + 150
+        qpos = [ld - 1 - (7 * t) % 1000 for t in range(T)]
+        idx, err = _topk_gpu(s, qpos, k)
+        assert err == 0
+        check_topk(idx, s, qpos, k)
+
+
+def test_topk_ties_straddle_slices():
+    # the K-th score is shared by positions in every slice of a long row: the lowest positions win
+    g = torch.Generator().manual_seed(10)
+    n = 40000
+    s = torch.randn(1, n, generator=g)
+    perm = torch.randperm(n, generator=g)
+    s[0, perm[:1000]] = 6.0
+    s[0, perm[1000:4000]] = 5.0
+    idx, err = _topk_gpu(s, [n - 1], 2048)
+    assert err == 0
+    check_topk(idx, s, [n - 1], 2048)
+    fives = torch.sort(perm[1000:4000]).values[:1048]
+    want = torch.sort(torch.cat([perm[:1000], fives])).values
+    assert idx[0].tolist() == want.tolist()
+
+
+def test_topk_skewed_and_equal_long_rows():
+    g = torch.Generator().manual_seed(11)
+    T, ld = 4, 120000
+    s = torch.randn(T, ld, generator=g)
+    s[0, :3000] += 10.0              # every selected score in the first slice
+    s[1, -2500:] += 10.0             # ... in the last slice
+    s[2] = 3.25                      # all equal: more ties than candidates fit
+    s[3] = torch.randint(0, 3, (ld,), generator=g).float()  # three values, heavy ties
+    qpos = [ld - 1, ld - 1, ld - 1, ld - 1]
+    idx, err = _topk_gpu(s, qpos, 2048)
+    assert err == 0
+    check_topk(idx, s, qpos, 2048)
+    assert idx[2].tolist() == list(range(2048))
+
+
+def test_topk_nan_in_long_row():
+    s = torch.randn(2, 100000)
+    s[1, 77777] = float("nan")
+    idx, err = _topk_gpu(s, [99999, 99999], 2048)
+    assert err & dsa.DEVERR_NAN_SCORE
+    check_topk(idx[:1], s[:1], [99999], 2048)
+
+
 def test_topk_nan_sets_error_word():
     s = torch.randn(1, 5000)
     s[0, 77] = float("nan")
