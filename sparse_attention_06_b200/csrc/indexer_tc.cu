@@ -6,10 +6,9 @@
 // with 64 indexer heads of 128 dims, bf16 queries, and bf16 keys or e4m3 keys with a per-token
 // scale (khat = code * scale; for scale > 0 the scale is applied after the head sum, which is the
 // same value).  bf16 keys multiply bf16 queries exactly as stored.  For e4m3 keys the product runs
-// in f16: each code is re-encoded by integer bit operations as the f16 holding code * 2^-8 (exact
-// for every finite code, subnormals included), the epilogue multiplies the per-token scale by 2^8,
-// and each query tile is converted bf16 -> f16 once, which is exact for |q| in [2^-14, 65504]
-// (smaller values keep an absolute error below 2^-25).
+// in f16: each pair of codes becomes two f16 by the hardware conversion (cvt.rn.f16x2.e4m3x2, exact:
+// every e4m3 value, subnormals included, is an f16), and each query tile is converted bf16 -> f16
+// once, which is exact for |q| in [2^-14, 65504] (smaller values keep an absolute error below 2^-25).
 //
 // Shape of the computation: per tile of 128 consecutive key positions (two 64-token pages of the
 // paged key cache) one tensor-core product D[128 keys, 64*NQ] = K[128 keys, 128] . Q[64*NQ, 128]^T
@@ -19,11 +18,18 @@
 // in-thread work of the epilogue.
 //
 // One persistent CTA per SM walks a contiguous range of the (query group, key tile) list.  Roles:
-//   warp 0      TMA producer: key pages and query tiles into 128B-swizzled shared memory
+//   warp 0      producer: looks up the block ids of the next 32 tiles at once (one lane per tile,
+//               the following batch already in flight), then issues the TMA copies of key pages
+//               and query tiles into 128B-swizzled shared memory and records each tile's block
+//               ids in a tile-info ring
 //   warp 1      TMEM allocation and the single thread that issues tcgen05.mma / tcgen05.commit
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator, ReLU, head sum, scale, score stores
-//   warps 6-9   (e4m3 keys only) convert the fp8 staging tile into the f16 operand ring and each
-//               query tile to f16 in place
+//   epilogue    4 warps (8 when 4 queries share a tile, each warp half of them): reads the tile
+//               info LOOK tiles ahead (and, for e4m3, starts a 4-byte cp.async of its key's scale
+//               then), then per tile: tcgen05.ld of the accumulator, ReLU, head sum, scale, score
+//               stores
+//   converter   (e4m3 keys only) converts the fp8 staging tile to f16 -- into tensor memory, where
+//               the MMA reads it as the A operand, when one query uses the tile (8 warps), else
+//               into the shared-memory operand ring (4 warps) -- and each query tile to f16 in place
 // Every wait is bounded (DSA_DEVERR_TIMEOUT); bad block ids and bad query metadata are flagged in
 // the device error word and skipped, never trapped.
 #include <cuda.h>
@@ -43,23 +49,45 @@ constexpr int kDim = 128;
 template <int NQ, bool FP8>
 struct Cfg {
   static constexpr int N = kHeads * NQ;                       // MMA N
-  static constexpr int OPS = FP8 ? (NQ == 1 ? 3 : 2) : (NQ == 1 ? 5 : 4);  // operand stages
-  static constexpr int STS = FP8 ? (NQ == 1 ? 6 : 4) : 0;     // fp8 staging stages
+  // e4m3 keys with one query per tile: the converted key tile goes to tensor memory and the MMA
+  // reads its A operand from there (the accumulators of N = 64 leave room for four A stages)
+  static constexpr bool TMEM_A = FP8 && NQ == 1;
+  static constexpr int OPS = TMEM_A ? 4 : FP8 ? 2 : (NQ == 1 ? 5 : 4);  // operand stages
+  static constexpr int STS = FP8 ? (NQ == 1 ? 8 : 4) : 0;     // fp8 staging stages
   static constexpr int QS = NQ == 1 ? 2 : 1;                  // query slots
+  static constexpr int TIS = NQ == 1 ? 24 : 16;               // tile-info ring entries
+  // Tiles (of its own) an epilogue warp reads ahead in the tile-info ring.  The producer runs at
+  // most STS + OPS + 2 tiles (e4m3) or OPS + 2 tiles (bf16) ahead of the epilogue's last finished
+  // tile, so the distance stays below that; only e4m3 needs it (its scale copies).
+  static constexpr int LOOK = FP8 ? (NQ == 1 ? 4 : 4) : 1;
   static constexpr int OP_BYTES = kTileKeys * kDim * 2;       // 32 KB bf16 key tile
   static constexpr int CHUNK_BYTES = kTileKeys * 128;         // one 64-dim column block
   static constexpr int ST_BYTES = kTileKeys * kDim;           // 16 KB fp8 key tile
   static constexpr int Q_BYTES = N * kDim * 2;
   static constexpr int Q_CHUNK = N * 128;
-  static constexpr int TMEM_COLS = 2 * N;
-  static constexpr int THREADS = FP8 ? 320 : 192;
+  static constexpr int A_COLS = kDim / 2;                     // TMEM columns of one f16 key tile
+  static constexpr int A_COL0 = 2 * N;                        // first A stage (TMEM_A)
+  static constexpr int TMEM_COLS = TMEM_A ? 512 : 2 * N;
+  // Epilogue: two sets of four warps (each set covers the 128 TMEM lanes).  With one query per
+  // tile the sets take alternate tiles (set s owns accumulator s); with four queries both sets
+  // take every tile, each scoring two of the queries.
+  static constexpr int EPI_WARPS = 8;
+  static constexpr bool EPI_ALT = NQ == 1;
+  static constexpr int EPI_NQ = EPI_ALT ? NQ : NQ / 2;       // queries per epilogue warp
+  static constexpr int EPI_ARRIVE = EPI_ALT ? 4 : 8;          // epilogue arrivals per tile
+  static constexpr int CONV_WARPS = FP8 ? 4 : 0;
+  static constexpr int CONV0 = 2 + EPI_WARPS;                 // first converter warp
+  static constexpr int THREADS = 32 * (CONV0 + CONV_WARPS);
   // shared-memory carve-up (offsets from a 1024-aligned base)
   static constexpr int OFF_OP = 0;
-  static constexpr int OFF_ST = OFF_OP + OPS * OP_BYTES;
+  static constexpr int OFF_ST = OFF_OP + (TMEM_A ? 0 : OPS * OP_BYTES);
   static constexpr int OFF_Q = OFF_ST + STS * ST_BYTES;
   static constexpr int OFF_W = OFF_Q + QS * Q_BYTES;
-  static constexpr int OFF_BAR = OFF_W + 4 * NQ * kHeads * 4;  // one copy of w per epilogue warp
-  static constexpr int NBAR = 2 * OPS + 2 * STS + 3 * QS + 4 + 1;
+  static constexpr int OFF_SC = OFF_W + EPI_WARPS * EPI_NQ * kHeads * 4;  // w, one copy per epilogue warp
+  static constexpr int OFF_PR = OFF_SC + (FP8 ? TIS * kTileKeys * 4 : 0);  // key scales of ring tiles
+  static constexpr int OFF_TI = OFF_PR + TIS * kTileKeys;                  // row present, per ring tile
+  static constexpr int OFF_BAR = OFF_TI + TIS * 8;                         // block ids of ring tiles
+  static constexpr int NBAR = 2 * OPS + 2 * STS + 3 * QS + 4 + 1 + 2 * TIS;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 64;
   static constexpr int SMEM = BYTES + 1024;  // slack for aligning the base
@@ -150,22 +178,27 @@ struct Walk {
   }
 };
 
-// Physical block of page `pg` (0/1) of tile `j` of a group, or -1 when the page holds no
-// visible key or its block id is outside the pool.
-__device__ __forceinline__ int page_block(const Params& p, const Group& G, int j, int pg, bool report) {
+// Raw block-table entry of page `pg` (0/1) of tile `j` of a group: -1 when the page holds no
+// visible key, -2 when its logical block is past the table.  Only the load; check_block() judges
+// the value when it is used, so that the load stays in flight until then.  A negative table entry
+// for a page with visible keys is an error like any other id outside the pool (it reads as -3).
+__device__ __forceinline__ int lookup_block(const Params& p, const Group& G, int j, int pg) {
   const int first = j * kTileKeys + pg * kPage;
-  if (first >= G.nmax) return -1;
+  if (G.tiles == 0 || first >= G.nmax) return -1;
   const int lblk = first / kPage;
-  if (lblk >= p.max_blocks) {
-    if (report) raise_error(p.err, DSA_DEVERR_BLOCK_ID);
+  if (lblk >= p.max_blocks) return -2;
+  const int b = p.block_table[(int64_t)G.req * p.max_blocks + lblk];
+  return b < 0 ? -3 : b;
+}
+
+// The physical block of a looked-up entry, or -1 (flagging entries outside the pool).
+__device__ __forceinline__ int check_block(const Params& p, int raw) {
+  if (raw == -1) return -1;
+  if (raw < 0 || raw >= p.num_blocks) {
+    raise_error(p.err, DSA_DEVERR_BLOCK_ID);
     return -1;
   }
-  const int blk = p.block_table[(int64_t)G.req * p.max_blocks + lblk];
-  if (blk < 0 || blk >= p.num_blocks) {
-    if (report) raise_error(p.err, DSA_DEVERR_BLOCK_ID);
-    return -1;
-  }
-  return blk;
+  return raw;
 }
 
 // Bounded wait that ignores the abort flag (used to drain in-flight copies when giving up).
@@ -173,25 +206,23 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* 
   mbar_wait(bar, parity, err, nullptr);
 }
 
-// Two e4m3 codes -> two f16 holding code * 2^-8, exactly.  An e4m3 code s.eeee.mmm has value
-// (1 + m/8) 2^(e-7) (or (m/8) 2^-6 when e = 0); its 7 magnitude bits placed at f16 bits 7..13 read
-// as (1 + m/8) 2^(e-15) (or, as an f16 subnormal, (m/8) 2^-14): the same value times 2^-8 in both
-// cases.  The sign moves from bit 7 to bit 15.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_times_2m8(uint32_t w, uint32_t byte_sel) {
-  const uint32_t x = __byte_perm(w, 0u, byte_sel);  // code a in bits 0..7, code b in bits 16..23
-  return ((x << 7) & 0x3F803F80u) | ((x << 8) & 0x80008000u);
+// Four e4m3 codes (one 32-bit word, lowest byte first) -> four f16 in two words, exactly, by the
+// hardware conversion.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\t"
+      "mov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
 
-// fp8 e4m3 x16 -> f16 x16, each value scaled by 2^-8 (exact)
+// fp8 e4m3 x16 -> f16 x16 (exact)
 __device__ __forceinline__ void e4m3x16_to_f16(const uint4& in, uint4& lo, uint4& hi) {
-  lo.x = e4m3x2_to_f16x2_times_2m8(in.x, 0x4140u);
-  lo.y = e4m3x2_to_f16x2_times_2m8(in.x, 0x4342u);
-  lo.z = e4m3x2_to_f16x2_times_2m8(in.y, 0x4140u);
-  lo.w = e4m3x2_to_f16x2_times_2m8(in.y, 0x4342u);
-  hi.x = e4m3x2_to_f16x2_times_2m8(in.z, 0x4140u);
-  hi.y = e4m3x2_to_f16x2_times_2m8(in.z, 0x4342u);
-  hi.z = e4m3x2_to_f16x2_times_2m8(in.w, 0x4140u);
-  hi.w = e4m3x2_to_f16x2_times_2m8(in.w, 0x4342u);
+  e4m3x4_to_f16x4(in.x, lo.x, lo.y);
+  e4m3x4_to_f16x4(in.y, lo.z, lo.w);
+  e4m3x4_to_f16x4(in.z, hi.x, hi.y);
+  e4m3x4_to_f16x4(in.w, hi.z, hi.w);
 }
 
 // bf16 x8 -> f16 x8 in place (16 bytes)
@@ -219,6 +250,9 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
   uint8_t* st_ring = smem + C::OFF_ST;
   uint8_t* q_slots = smem + C::OFF_Q;
   float* w_s = reinterpret_cast<float*>(smem + C::OFF_W);
+  float* sc_ring = reinterpret_cast<float*>(smem + C::OFF_SC);  // [TIS][128] (e4m3) key scales
+  uint8_t* pr_ring = smem + C::OFF_PR;                           // [TIS][128] row's page present
+  int2* ti_ring = reinterpret_cast<int2*>(smem + C::OFF_TI);     // [TIS] block ids of the pages
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* op_full = bars;
   uint64_t* op_empty = op_full + C::OPS;
@@ -230,6 +264,8 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
   uint64_t* acc_full = q_ready + C::QS;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* mma_done = acc_empty + 2;
+  uint64_t* ti_full = mma_done + 1;     // [TIS] tile info (and scales) in place
+  uint64_t* ti_empty = ti_full + C::TIS;  // [TIS] tile info read by every epilogue warp
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
   unsigned long long* total_tiles = reinterpret_cast<unsigned long long*>(smem + C::OFF_MISC + 16);
@@ -239,23 +275,27 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
 
   if (tid == 0) {
     for (int i = 0; i < C::OPS; ++i) {
-      mbar_init(&op_full[i], FP8 ? 128 : 1);
+      mbar_init(&op_full[i], FP8 ? C::CONV_WARPS : 1);
       mbar_init(&op_empty[i], 1);
     }
     for (int i = 0; i < C::STS; ++i) {
       mbar_init(&st_full[i], 1);
-      mbar_init(&st_empty[i], 128);
+      mbar_init(&st_empty[i], C::CONV_WARPS);
     }
     for (int i = 0; i < C::QS; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
-      mbar_init(&q_ready[i], 128);
+      mbar_init(&q_ready[i], C::CONV_WARPS);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
+      mbar_init(&acc_empty[i], C::EPI_ARRIVE);
     }
     mbar_init(mma_done, 1);
+    for (int i = 0; i < C::TIS; ++i) {
+      mbar_init(&ti_full[i], 1);
+      mbar_init(&ti_empty[i], C::EPI_ARRIVE);
+    }
     *abort_flag = 0;
     *total_tiles = 0ull;
     fence_mbar_init();
@@ -281,54 +321,99 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
   const int64_t hi = N * (blockIdx.x + 1) / gridDim.x;
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0 && lo < hi) {
-      prefetch_tmap(&kmap);
-      prefetch_tmap(&qmap);
+    // ------------------------------------------------------------------ producer
+    if (lo < hi) {
+      if (lane == 0) {
+        prefetch_tmap(&kmap);
+        prefetch_tmap(&qmap);
+      }
+      // Every lane runs the same walk; lane l keeps tile l of each batch of 32 and loads its two
+      // block ids.  The next batch is looked up before the current one is issued.
       Walk<NQ> W;
       W.init(p, lo, hi);
-      int grp, j, last = -1, m = -1;
+      int n_cnt = 0, n_grp = -1, n_r0 = -1, n_r1 = -1;
+      auto fetch = [&]() {
+        n_cnt = 0;
+        n_grp = -1;
+        int mj = 0;
+        Group mG{0, 0, 0};
+        for (int l = 0; l < 32; ++l) {
+          int g, j;
+          if (!W.next(p, g, j)) break;
+          if (lane == l) {
+            n_grp = g;
+            mj = j;
+            mG = W.G;
+          }
+          ++n_cnt;
+        }
+        n_r0 = n_grp >= 0 ? lookup_block(p, mG, mj, 0) : -1;
+        n_r1 = n_grp >= 0 ? lookup_block(p, mG, mj, 1) : -1;
+      };
+      fetch();
+      int last = -1, m = -1;
       int64_t i = 0;
       bool ok = true;
-      while (ok && W.next(p, grp, j)) {
-        if (grp != last) {
-          last = grp;
-          ++m;
-          const int slot = m % C::QS, use = m / C::QS;
-          if (use >= 1 && !(ok = mbar_wait(&q_empty[slot], (use - 1) & 1, p.err, abort_flag))) break;
-          mbar_arrive_expect_tx(&q_full[slot], C::Q_BYTES);
-          uint8_t* qd = q_slots + slot * C::Q_BYTES;
-          tma_load_2d(qd, &qmap, &q_full[slot], 0, grp * NQ * kHeads);
-          tma_load_2d(qd + C::Q_CHUNK, &qmap, &q_full[slot], 64, grp * NQ * kHeads);
-        }
-        const int b0 = page_block(p, W.G, j, 0, true);
-        const int b1 = page_block(p, W.G, j, 1, true);
-        if (FP8) {
-          const int s = (int)(i % C::STS), use = (int)(i / C::STS);
-          if (use >= 1 && !(ok = mbar_wait(&st_empty[s], (use - 1) & 1, p.err, abort_flag))) break;
-          const uint32_t bytes = (b0 >= 0 ? 8192u : 0u) + (b1 >= 0 ? 8192u : 0u);
-          mbar_arrive_expect_tx(&st_full[s], bytes);
-          uint8_t* dst = st_ring + s * C::ST_BYTES;
-          if (b0 >= 0) tma_load_2d(dst, &kmap, &st_full[s], 0, b0 * kPage);
-          if (b1 >= 0) tma_load_2d(dst + 8192, &kmap, &st_full[s], 0, b1 * kPage);
-        } else {
-          const int s = (int)(i % C::OPS), use = (int)(i / C::OPS);
-          if (use >= 1 && !(ok = mbar_wait(&op_empty[s], (use - 1) & 1, p.err, abort_flag))) break;
-          const uint32_t bytes = (b0 >= 0 ? 16384u : 0u) + (b1 >= 0 ? 16384u : 0u);
-          mbar_arrive_expect_tx(&op_full[s], bytes);
-          uint8_t* dst = op_ring + s * C::OP_BYTES;
-          if (b0 >= 0) {
-            tma_load_2d(dst, &kmap, &op_full[s], 0, b0 * kPage);
-            tma_load_2d(dst + C::CHUNK_BYTES, &kmap, &op_full[s], 64, b0 * kPage);
+      while (ok && n_cnt > 0) {
+        const int cnt = n_cnt, my_grp = n_grp, r0 = n_r0, r1 = n_r1;
+        fetch();
+        for (int l = 0; l < cnt; ++l) {
+          const int grp = __shfl_sync(0xFFFFFFFFu, my_grp, l);
+          const int raw0 = __shfl_sync(0xFFFFFFFFu, r0, l);
+          const int raw1 = __shfl_sync(0xFFFFFFFFu, r1, l);
+          if (lane == 0) {
+            const int b0 = check_block(p, raw0);
+            const int b1 = check_block(p, raw1);
+            {
+              // tile info for the epilogue: the block ids of the tile's pages (-1: absent).  It is
+              // published before any wait of this tile below, which depend on the epilogue.
+              const int c = (int)(i % C::TIS), cu = (int)(i / C::TIS);
+              if (cu >= 1 && !(ok = mbar_wait(&ti_empty[c], (cu - 1) & 1, p.err, abort_flag))) goto issued;
+              ti_ring[c] = make_int2(b0, b1);
+              mbar_arrive(&ti_full[c]);
+            }
+            if (grp != last) {
+              const int mm = m + 1;  // m counts the query tiles issued so far
+              const int slot = mm % C::QS, use = mm / C::QS;
+              if (use >= 1 && !(ok = mbar_wait(&q_empty[slot], (use - 1) & 1, p.err, abort_flag))) goto issued;
+              mbar_arrive_expect_tx(&q_full[slot], C::Q_BYTES);
+              uint8_t* qd = q_slots + slot * C::Q_BYTES;
+              tma_load_2d(qd, &qmap, &q_full[slot], 0, grp * NQ * kHeads);
+              tma_load_2d(qd + C::Q_CHUNK, &qmap, &q_full[slot], 64, grp * NQ * kHeads);
+              m = mm;
+              last = grp;
+            }
+            {
+              if (FP8) {
+                const int s = (int)(i % C::STS), use = (int)(i / C::STS);
+                if (use >= 1 && !(ok = mbar_wait(&st_empty[s], (use - 1) & 1, p.err, abort_flag))) goto issued;
+                mbar_arrive_expect_tx(&st_full[s], (b0 >= 0 ? 8192u : 0u) + (b1 >= 0 ? 8192u : 0u));
+                uint8_t* dst = st_ring + s * C::ST_BYTES;
+                if (b0 >= 0) tma_load_2d(dst, &kmap, &st_full[s], 0, b0 * kPage);
+                if (b1 >= 0) tma_load_2d(dst + 8192, &kmap, &st_full[s], 0, b1 * kPage);
+              } else {
+                const int s = (int)(i % C::OPS), use = (int)(i / C::OPS);
+                if (use >= 1 && !(ok = mbar_wait(&op_empty[s], (use - 1) & 1, p.err, abort_flag))) goto issued;
+                mbar_arrive_expect_tx(&op_full[s], (b0 >= 0 ? 16384u : 0u) + (b1 >= 0 ? 16384u : 0u));
+                uint8_t* dst = op_ring + s * C::OP_BYTES;
+                if (b0 >= 0) {
+                  tma_load_2d(dst, &kmap, &op_full[s], 0, b0 * kPage);
+                  tma_load_2d(dst + C::CHUNK_BYTES, &kmap, &op_full[s], 64, b0 * kPage);
+                }
+                if (b1 >= 0) {
+                  tma_load_2d(dst + 8192, &kmap, &op_full[s], 0, b1 * kPage);
+                  tma_load_2d(dst + C::CHUNK_BYTES + 8192, &kmap, &op_full[s], 64, b1 * kPage);
+                }
+              }
+            }
+            ++i;
+          issued:;
           }
-          if (b1 >= 0) {
-            tma_load_2d(dst + 8192, &kmap, &op_full[s], 0, b1 * kPage);
-            tma_load_2d(dst + C::CHUNK_BYTES + 8192, &kmap, &op_full[s], 64, b1 * kPage);
-          }
+          ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+          if (!ok) break;
         }
-        ++i;
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         // give up: let the copies already issued land before the CTA's memory goes away
         for (int s = 0; s < C::OPS && !FP8; ++s)
           if (i > s) drain_wait(&op_full[s], (uint32_t)(((i - 1 - s) / C::OPS) & 1), p.err);
@@ -362,18 +447,31 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
         tc_fence_after();
         // 8 MMAs of K = 16: two 64-dim column blocks, four K steps of 32 bytes each (the
         // descriptor's start-address field counts 16-byte units)
-        const uint64_t ad = sw128_desc(smem_u32(op_ring + s * C::OP_BYTES), 16, 1024);
         const uint64_t bd = sw128_desc(smem_u32(q_slots + slot * C::Q_BYTES), 16, 1024);
         const uint32_t d = tmem_base + (uint32_t)(a * C::N);
         constexpr uint64_t ac = C::CHUNK_BYTES >> 4, bc = C::Q_CHUNK >> 4;
-        umma_ss<0>(d, ad, bd, idesc);
-        umma_ss<1>(d, ad + 2, bd + 2, idesc);
-        umma_ss<1>(d, ad + 4, bd + 4, idesc);
-        umma_ss<1>(d, ad + 6, bd + 6, idesc);
-        umma_ss<1>(d, ad + ac, bd + bc, idesc);
-        umma_ss<1>(d, ad + ac + 2, bd + bc + 2, idesc);
-        umma_ss<1>(d, ad + ac + 4, bd + bc + 4, idesc);
-        umma_ss<1>(d, ad + ac + 6, bd + bc + 6, idesc);
+        if (C::TMEM_A) {
+          // A = the f16 key tile in tensor memory: one K step of 16 dims = 8 columns
+          const uint32_t at = tmem_base + (uint32_t)(C::A_COL0 + s * C::A_COLS);
+          umma_ts<0>(d, at, bd, idesc);
+          umma_ts<1>(d, at + 8, bd + 2, idesc);
+          umma_ts<1>(d, at + 16, bd + 4, idesc);
+          umma_ts<1>(d, at + 24, bd + 6, idesc);
+          umma_ts<1>(d, at + 32, bd + bc, idesc);
+          umma_ts<1>(d, at + 40, bd + bc + 2, idesc);
+          umma_ts<1>(d, at + 48, bd + bc + 4, idesc);
+          umma_ts<1>(d, at + 56, bd + bc + 6, idesc);
+        } else {
+          const uint64_t ad = sw128_desc(smem_u32(op_ring + s * C::OP_BYTES), 16, 1024);
+          umma_ss<0>(d, ad, bd, idesc);
+          umma_ss<1>(d, ad + 2, bd + 2, idesc);
+          umma_ss<1>(d, ad + 4, bd + 4, idesc);
+          umma_ss<1>(d, ad + 6, bd + 6, idesc);
+          umma_ss<1>(d, ad + ac, bd + bc, idesc);
+          umma_ss<1>(d, ad + ac + 2, bd + bc + 2, idesc);
+          umma_ss<1>(d, ad + ac + 4, bd + bc + 4, idesc);
+          umma_ss<1>(d, ad + ac + 6, bd + bc + 6, idesc);
+        }
         mma_commit(&op_empty[s]);
         mma_commit(&acc_full[a]);
         ++i;
@@ -382,64 +480,69 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
       mma_commit(mma_done);
       drain_wait(mma_done, 0, p.err);
     }
-  } else if (warp < 6) {
+  } else if (warp < C::CONV0) {
     // ------------------------------------------------------------------ epilogue
+    const int ew = warp - 2;                   // epilogue warp
+    const int eset = ew >> 2;                  // its set
     const int quarter = warp & 3;              // TMEM lanes this warp may access
+    const int q0 = C::EPI_ALT ? 0 : eset * C::EPI_NQ;  // first query of the group this warp scores
+    const int t0 = C::EPI_ALT ? eset : 0;      // first tile of this warp, then every tstep-th
+    constexpr int tstep = C::EPI_ALT ? 2 : 1;
     const int r = quarter * 32 + lane;         // key row of the tile
-    float* w_mine = w_s + (warp - 2) * NQ * kHeads;  // this warp's copy of the group's w
-    const int pg = r >> 6;                           // page of the tile holding this row
-    // Tiles are looked up ahead of their accumulator: the block id two tiles ahead and the e4m3
-    // scale one tile ahead, so that neither global load is waited on in the tile that issued it.
+    float* w_mine = w_s + ew * C::EPI_NQ * kHeads;  // this warp's copy of its queries' w
+    const int64_t ntl = hi - lo;               // tiles of this CTA
+    bool ok = true;
+    // Tile `it` seen C::LOOK of this warp's tiles ahead: note whether this row's page exists and
+    // (e4m3) start the copy of the row's key scale; each thread reads back only what it wrote
+    // itself, after its own cp.async group of that tile has completed.  One group is committed per
+    // tile of this warp (empty past the end) so that the group count stays in step.
+    auto look = [&](int64_t it) {
+      if (it < ntl && ok) {
+        const int c = (int)(it % C::TIS);
+        ok = warp_wait(&ti_full[c], (uint32_t)((it / C::TIS) & 1), p.err, abort_flag);
+        if (ok) {
+          const int2 blk = ti_ring[c];
+          const int b = r < kPage ? blk.x : blk.y;
+          pr_ring[c * kTileKeys + r] = b >= 0 ? 1 : 0;
+          if (FP8 && b >= 0)
+            cp_async_4(smem_u32(sc_ring + c * kTileKeys + r), p.key_scale + (int64_t)b * kPage + (r & (kPage - 1)));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ti_empty[c]);
+        }
+      }
+      cp_async_commit();
+    };
+#pragma unroll 1
+    for (int d = 0; d < C::LOOK; ++d) look(t0 + (int64_t)d * tstep);
     Walk<NQ> W;
     W.init(p, lo, hi);
-    int g0 = -1, j0 = 0, g1 = -1, j1 = 0, g2 = -1, j2 = 0;
-    Group G0{0, 0, 0}, G1{0, 0, 0}, G2{0, 0, 0};
-    int b0 = -1, b1 = -1, b2 = -1;
-    float sc0 = 1.0f, sc1 = 1.0f;
-    if (W.next(p, g1, j1)) {
-      G1 = W.G;
-      b1 = page_block(p, G1, j1, pg, false);
-      if (W.next(p, g2, j2)) {
-        G2 = W.G;
-        b2 = page_block(p, G2, j2, pg, false);
-      } else {
-        g2 = -1;
-      }
-      if (FP8 && b1 >= 0) sc1 = 256.0f * p.key_scale[(int64_t)b1 * kPage + (r & 63)];
-    } else {
-      g1 = -1;
-    }
-    int last = -1;
-    int npos[NQ];
+    int grp, j, last = -1;
+    int npos[C::EPI_NQ];
     int64_t i = 0;
-    while (g1 >= 0) {
-      // rotate: the tile to finish now is the one looked up last iteration
-      g0 = g1; j0 = j1; G0 = G1; b0 = b1; sc0 = sc1;
-      g1 = g2; j1 = j2; G1 = G2; b1 = b2;
-      sc1 = 1.0f;
-      if (g1 >= 0 && FP8 && b1 >= 0) sc1 = 256.0f * p.key_scale[(int64_t)b1 * kPage + (r & 63)];  // undo 2^-8
-      if (g1 >= 0 && W.next(p, g2, j2)) {
-        G2 = W.G;
-        b2 = page_block(p, G2, j2, pg, false);
-      } else {
-        g2 = -1;
+    while (ok && W.next(p, grp, j)) {
+      if ((i & (tstep - 1)) != t0) {  // the other set's tile
+        ++i;
+        continue;
       }
-      if (g0 != last) {
+      if (grp != last) {
         __syncwarp();
-        for (int e = lane; e < NQ * kHeads; e += 32) w_mine[e] = p.w[(int64_t)g0 * NQ * kHeads + e];
+        for (int e = lane; e < C::EPI_NQ * kHeads; e += 32) w_mine[e] = p.w[(int64_t)(grp * NQ + q0) * kHeads + e];
         __syncwarp();
 #pragma unroll
-        for (int qi = 0; qi < NQ; ++qi) npos[qi] = p.q_pos[g0 * NQ + qi] + 1;
-        last = g0;
+        for (int qi = 0; qi < C::EPI_NQ; ++qi) npos[qi] = p.q_pos[grp * NQ + q0 + qi] + 1;
+        last = grp;
       }
+      cp_async_wait<C::LOOK - 1>();  // this tile's group (committed LOOK tiles ago) has landed
+      const int c = (int)(i % C::TIS);
+      const bool present = pr_ring[c * kTileKeys + r] != 0;
+      const float scale = FP8 ? sc_ring[c * kTileKeys + r] : 1.0f;
       const int a = (int)(i & 1), use = (int)(i >> 1);
       if (!warp_wait(&acc_full[a], use & 1, p.err, abort_flag)) break;
       tc_fence_after();
-      const int s = j0 * kTileKeys + r;
-      const float scale = FP8 ? sc0 : 1.0f;
-      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * C::N);
+      const int s = j * kTileKeys + r;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * C::N + q0 * kHeads);
 #pragma unroll
-      for (int qi = 0; qi < NQ; ++qi) {
+      for (int qi = 0; qi < C::EPI_NQ; ++qi) {
         uint32_t v[64];
         tmem_ld16(tbase + qi * 64 + 0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
         tmem_ld16(tbase + qi * 64 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
@@ -447,25 +550,32 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
         tmem_ld16(tbase + qi * 64 + 48, *reinterpret_cast<uint32_t(*)[16]>(&v[48]));
         tmem_wait_ld();
         const float4* w4 = reinterpret_cast<const float4*>(w_mine + qi * kHeads);
-        float acc0 = 0.0f, acc1 = 0.0f;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
 #pragma unroll
         for (int h4 = 0; h4 < 16; ++h4) {
           const float4 wv = w4[h4];
-          acc0 = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * h4 + 0]), 0.0f), acc0);
-          acc1 = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * h4 + 1]), 0.0f), acc1);
-          acc0 = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * h4 + 2]), 0.0f), acc0);
-          acc1 = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * h4 + 3]), 0.0f), acc1);
+          float* ac = acc + (h4 & 1) * 4;
+          ac[0] = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * h4 + 0]), 0.0f), ac[0]);
+          ac[1] = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * h4 + 1]), 0.0f), ac[1]);
+          ac[2] = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * h4 + 2]), 0.0f), ac[2]);
+          ac[3] = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * h4 + 3]), 0.0f), ac[3]);
         }
-        if (b0 >= 0 && s < npos[qi]) p.scores[(int64_t)(g0 * NQ + qi) * p.ld + s] = (acc0 + acc1) * scale;
+        const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        if (present && s < npos[qi]) p.scores[(int64_t)(grp * NQ + q0 + qi) * p.ld + s] = sum * scale;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[a]);
+      look(i + (int64_t)C::LOOK * tstep);  // after this tile is released, so that the producer can get there
       ++i;
     }
+    cp_async_wait_all();  // no copy may land after the CTA's shared memory is released
   } else if (FP8) {
-    // ------------------------------------------------------------------ fp8 -> bf16 converter
-    const int ct = tid - 192;  // 0..127
+    // ------------------------------------------------------------------ fp8 -> f16 converter
+    const int cw = warp - C::CONV0;  // 0 .. CONV_WARPS-1
+    const int ct = tid - 32 * C::CONV0;
     Walk<NQ> W;
     W.init(p, lo, hi);
     int grp, j, last = -1, m = -1;
@@ -478,32 +588,63 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
         const int slot = m % C::QS;
         if (!warp_wait(&q_full[slot], (m / C::QS) & 1, p.err, abort_flag)) break;
         uint8_t* q = q_slots + slot * C::Q_BYTES;
-        for (int off = ct * 16; off < C::Q_BYTES; off += 128 * 16)
+        for (int off = ct * 16; off < C::Q_BYTES; off += 32 * C::CONV_WARPS * 16)
           *reinterpret_cast<uint4*>(q + off) = bf16x8_to_f16(*reinterpret_cast<const uint4*>(q + off));
         fence_proxy_async_smem();
-        mbar_arrive(&q_ready[slot]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_ready[slot]);
       }
       const int s8 = (int)(i % C::STS), u8 = (int)(i / C::STS);
       if (!warp_wait(&st_full[s8], u8 & 1, p.err, abort_flag)) break;
       const int so = (int)(i % C::OPS), uo = (int)(i / C::OPS);
       if (uo >= 1 && !warp_wait(&op_empty[so], (uo - 1) & 1, p.err, abort_flag)) break;
       const uint8_t* src = st_ring + s8 * C::ST_BYTES;
-      uint8_t* dst = op_ring + so * C::OP_BYTES;
-#pragma unroll 2
-      for (int k = 0; k < 8; ++k) {
-        const int piece = ct + 128 * k;  // 16-byte piece of the fp8 tile: row piece/8, column piece%8
-        const int row = piece >> 3, c = piece & 7;
-        const uint4 in = *reinterpret_cast<const uint4*>(src + row * 128 + c * 16);
-        uint4 lo4, hi4;
-        e4m3x16_to_f16(in, lo4, hi4);
-        uint8_t* chunk = dst + (c >> 2) * C::CHUNK_BYTES;
-        const uint32_t p0 = (uint32_t)((c & 3) * 2);
-        *reinterpret_cast<uint4*>(chunk + sw128_offset(row, p0)) = lo4;
-        *reinterpret_cast<uint4*>(chunk + sw128_offset(row, p0 + 1)) = hi4;
+      if (C::TMEM_A) {
+        // this thread: key row `row` (its TMEM lane); the staging tile is 128B-swizzled, so the
+        // lanes of a warp read distinct banks
+        tc_fence_after();
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t ta = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(C::A_COL0 + so * C::A_COLS);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // dims [64 h, 64 h + 64) -> 32 columns
+          uint32_t f[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 in = *reinterpret_cast<const uint4*>(src + sw128_offset(row, h * 4 + c));
+            uint4 lo4, hi4;
+            e4m3x16_to_f16(in, lo4, hi4);
+            f[8 * c + 0] = lo4.x; f[8 * c + 1] = lo4.y; f[8 * c + 2] = lo4.z; f[8 * c + 3] = lo4.w;
+            f[8 * c + 4] = hi4.x; f[8 * c + 5] = hi4.y; f[8 * c + 6] = hi4.z; f[8 * c + 7] = hi4.w;
+          }
+          tmem_st16(ta + h * 32, *reinterpret_cast<uint32_t(*)[16]>(&f[0]));
+          tmem_st16(ta + h * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&f[16]));
+        }
+        tmem_wait_st();
+        tc_fence_before();
+      } else {
+        // 8 codes -> one 16-byte chunk of the swizzled operand: the 8 threads of a quarter-warp
+        // fill the 8 chunks of one 128-byte row, so the stores hit distinct banks
+        uint8_t* dst = op_ring + so * C::OP_BYTES;
+        constexpr int kSteps = (kTileKeys * kDim / 8) / (32 * (C::CONV_WARPS > 0 ? C::CONV_WARPS : 1));
+#pragma unroll 4
+        for (int k = 0; k < kSteps; ++k) {
+          const int piece = ct + 32 * C::CONV_WARPS * k;  // 8-byte piece: row piece/16, codes 8 (piece%16) ..
+          const int row = piece >> 4, c8 = piece & 15;
+          const uint2 in = *reinterpret_cast<const uint2*>(src + row * 128 + c8 * 8);
+          uint4 o;
+          e4m3x4_to_f16x4(in.x, o.x, o.y);
+          e4m3x4_to_f16x4(in.y, o.z, o.w);
+          *reinterpret_cast<uint4*>(dst + (c8 >> 3) * C::CHUNK_BYTES + sw128_offset(row, c8 & 7)) = o;
+        }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&op_full[so]);
-      mbar_arrive(&st_empty[s8]);
+      (void)cw;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&op_full[so]);
+        mbar_arrive(&st_empty[s8]);
+      }
       ++i;
     }
   }
@@ -524,7 +665,7 @@ cudaError_t launch_impl(const IndexerArgs& a, int num_sms, cudaStream_t s) {
   const uint64_t rows = (uint64_t)a.keys.num_blocks * kPage;
   bool ok;
   if (FP8)
-    ok = encode_tmap_2d(&kmap, a.keys.data, 1, kDim, rows, kDim, 128, kPage, false);
+    ok = encode_tmap_2d(&kmap, a.keys.data, 1, kDim, rows, kDim, 128, kPage, C::TMEM_A);
   else
     ok = encode_tmap_2d(&kmap, a.keys.data, 2, kDim, rows, kDim * 2, 64, kPage, true);
   ok = ok && encode_tmap_2d(&qmap, a.q, 2, kDim, (uint64_t)a.batch.num_queries * kHeads, kDim * 2, 64,
