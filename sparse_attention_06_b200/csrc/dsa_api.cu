@@ -256,7 +256,8 @@ static dsa_status mla_common(bool decode, const void* q, int32_t q_dtype, int32_
   MlaArgs a{q, q_dtype, H, d_v, d_rope, *latent, *batch, idx, k, softmax_scale, out, lse,
             workspace, workspace_bytes, err};
   const bool tc_shape = H == 128 && d_v == 512 && d_rope == 64 && q_dtype == DSA_BF16 &&
-                        latent->block_size == 64 && aligned16(q) && aligned16(out);
+                        latent->block_size == 64 && aligned16(q) && aligned16(out) &&
+                        aligned16(latent->data);
   cudaError_t e;
   int kernels = 1;
   if (tc_shape) {

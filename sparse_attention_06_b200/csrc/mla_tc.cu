@@ -20,9 +20,14 @@
 // With several key splits per query each unit writes (O / l, LSE) partials that a small combine
 // kernel merges: O = sum_sp exp(LSE_sp - LSE) O_sp, LSE = log sum_sp exp(LSE_sp).
 //
-// Roles (288 threads): warps 0-3 gather rows with cp.async and write Q into tensor memory (warp
-// 0 lane 0 also loads Q's shared-memory part by TMA), warp 4 owns tensor memory and issues the
-// MMAs, warps 5-8 run the softmax and the epilogue (one head row per thread).
+// Roles (288 threads): warps 0-3 look up the rows of their 16 keys per tile and gather them with
+// TMA (tile::gather4: four rows x 128 bytes per instruction, 128B-swizzled by the copy itself;
+// unused slots point past the pool and read as zeros), and write Q into tensor memory (warp 0
+// lane 0 also loads Q's shared-memory part by TMA); warp 4 owns tensor memory and issues the
+// Q K^T products; warps 5-8 run the softmax and the epilogue (one head row per thread); warp 9
+// issues the P V products.  One thread issues a tensor-core instruction about every 60 cycles,
+// so the two product chains get separate issuing threads: the Q K^T chain of the next tile does
+// not hold back P V, which frees the row-ring stage for the next gather.
 // All waits are bounded; bad indices / block ids set the device error word and are skipped.
 #include <cuda.h>
 #include <math.h>
@@ -31,8 +36,8 @@
 #include "internal.h"
 
 namespace dsa {
-
 namespace {
+
 
 constexpr int kH = 128;         // heads (MMA M)
 constexpr int kDqk = 576;       // latent + rope
@@ -45,7 +50,8 @@ constexpr int kPage = 64;
 constexpr int kStages = 2;      // gathered-row ring
 constexpr int kGatherWarps = 4;
 constexpr int kKeysPerWarp = kTile / kGatherWarps;  // 16
-constexpr int kThreads = 32 * (kGatherWarps + 1 + 4);
+constexpr int kPvWarp = kGatherWarps + 5;                 // issues the P V products
+constexpr int kThreads = 32 * (kGatherWarps + 1 + 4 + 1);
 
 constexpr int Q_CHUNK = kH * 128;                            // 16 KB: 128 head rows x 64 dims
 constexpr int QS_BYTES = (kChunks - kTmemQChunks) * Q_CHUNK; // 48 KB of Q in shared memory
@@ -80,6 +86,7 @@ struct Params {
   float* part_o;                 // [T, nsplit, 128, 512] (several splits)
   float* part_lse;               // [T, nsplit, 128]
   int64_t num_blocks;
+  int32_t oob_row;               // first row past the pool (gathered as zeros)
   int T, k, ks, nsplit, num_reqs, max_blocks, max_context;
   float scale_log2;              // softmax scale * log2(e)
   int* err;
@@ -144,7 +151,8 @@ __device__ __forceinline__ int unit_tiles(const Params& p, int sp) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    mla_tc_kernel(const __grid_constant__ CUtensorMap qmap, const Params p) {
+    mla_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap lmap,
+                  const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_s = smem + OFF_Q;
@@ -177,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 32 * kGatherWarps + 1);
     mbar_init(q_empty, 1);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&k_full[i], 32 * kGatherWarps);
+      mbar_init(&k_full[i], kGatherWarps);
       mbar_init(&k_empty[i], 1);
       mbar_init(&m_full[i], kGatherWarps);
     }
@@ -185,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(s_empty, 4);
     mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
-    mbar_init(mma_fin, 1);
+    mbar_init(mma_fin, 2);  // both issuing threads
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -269,99 +277,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         ps_j = ps_j1;
         ps_j1 = ps_j2;
         blk_j = blk_j1;
-        const uint32_t stage_u32 = smem_u32(k_ring + s * K_BYTES);
-        // 16 rows x 72 pieces of 16 bytes = 36 per lane; 32 consecutive pieces per step
-#pragma unroll 4
-        for (int r = 0; r < 36; ++r) {
-          const int piece = lane + 32 * r;
-          const int kk = piece / 72, q16 = piece % 72;
-          const int64_t rw = __shfl_sync(0xFFFFFFFFu, row, kk);
-          const int key = gw * kKeysPerWarp + kk;
-          const char* src = reinterpret_cast<const char*>(p.latent) + (rw >= 0 ? rw : 0) * (kDqk * 2) + q16 * 16;
-          cp_async_16(stage_u32 + (q16 >> 3) * K_CHUNK + sw128_offset(key, q16 & 7), src, rw >= 0 ? 16u : 0u);
+        // this warp's 16 rows: four gather4 groups of four rows x nine 64-dim column blocks
+        const int32_t rc = row >= 0 ? (int32_t)row : p.oob_row;
+        uint8_t* stage = k_ring + s * K_BYTES + gw * kKeysPerWarp * 128;
+        if (lane == 0) mbar_arrive_expect_tx(&k_full[s], kKeysPerWarp * kDqk * 2);
+#pragma unroll
+        for (int g4 = 0; g4 < kKeysPerWarp / 4; ++g4) {
+          const int32_t r0 = __shfl_sync(0xFFFFFFFFu, rc, 4 * g4 + 0);
+          const int32_t r1 = __shfl_sync(0xFFFFFFFFu, rc, 4 * g4 + 1);
+          const int32_t r2 = __shfl_sync(0xFFFFFFFFu, rc, 4 * g4 + 2);
+          const int32_t r3 = __shfl_sync(0xFFFFFFFFu, rc, 4 * g4 + 3);
+          if (lane == 0) {
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c)
+              tma_gather4(stage + c * K_CHUNK + g4 * 512, &lmap, &k_full[s], c * 64, r0, r1, r2, r3);
+          }
         }
-        cp_async_mbar_arrive_noinc(&k_full[s]);
       }
     }
-    // let every copy this thread issued land before the CTA may exit
-    cp_async_wait_all();
+    if (!ok && lane == 0) {
+      // gave up: the row copies of the last use of each stage must land before the CTA exits
+      for (int t = gi - 1; t >= 0 && t >= gi - kStages; --t)
+        mbar_wait(&k_full[t % kStages], (uint32_t)((t / kStages) & 1), p.err, nullptr);
+    }
   } else if (warp == kGatherWarps) {
-    // ------------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------------ Q K^T issuer
     if (lane == 0) {
       const uint32_t idesc_s = idesc_f16(1u, 0u, 128u, (uint32_t)kTile);  // S: B K-major
-      const uint32_t idesc_o = idesc_f16(1u, 1u, 128u, (uint32_t)kHalf);  // O: B (V) MN-major
       int gi = 0, ui = 0;
       bool ok = true;
       const uint64_t qd = sw128_desc(smem_u32(q_s), 16, 1024);
-      // P [128 x 64] K-major, no swizzle: 8x16-byte core matrices 128 B apart along K and 1024 B
-      // apart along M; one K step (16 keys) is two core matrices = 256 bytes
-      const uint64_t pd = noswz_desc(smem_u32(p_s), 128, 1024);
-      const uint32_t d_s = tmem + TM_S, d_o = tmem + TM_O, a_q = tmem + TM_Q;
+      const uint32_t d_s = tmem + TM_S, a_q = tmem + TM_Q;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
         int t, sp, v;
         unit_coords(p, u, t, sp, v);
         const int ntiles = unit_tiles(p, sp);
         if (!(ok = mbar_wait(q_full, ui & 1, p.err, abort_flag))) break;
         if (ntiles == 0) mma_commit(q_empty);
-        // Issue whichever is ready: P V of the oldest finished softmax first (it frees a ring stage
-        // and lets the softmax move on), else the next tile's Q K^T.
-        int ns = 0, np = 0;
-        long long last = clock64();
-        while (np < ntiles) {
-          bool did = false;
-          if (np < ns) {
-            const int g = gi + np, s = g % kStages;
-            if (mbar_try_wait(p_full, g & 1)) {
-              // O_v += P V_v; V is MN-major 128B-swizzled: 64-dim blocks K_CHUNK apart, 8-row
-              // groups 1024 B apart, one K step (16 rows) = 2048 bytes
-              tc_fence_after();
-              const uint64_t vd = sw128_desc(smem_u32(k_ring + s * K_BYTES) + (uint32_t)(v * 4 * K_CHUNK), K_CHUNK, 1024);
-              if (np > 0)
-                umma_ss<1>(d_o, pd, vd, idesc_o);
-              else
-                umma_ss<0>(d_o, pd, vd, idesc_o);
-              umma_ss<1>(d_o, pd + 16, vd + 128, idesc_o);
-              umma_ss<1>(d_o, pd + 32, vd + 256, idesc_o);
-              umma_ss<1>(d_o, pd + 48, vd + 384, idesc_o);
-              mma_commit(pv_done);
-              mma_commit(&k_empty[s]);
-              ++np;
-              did = true;
-            }
-          }
-          if (!did && ns < ntiles) {
-            const int g = gi + ns, s = g % kStages;
-            if (mbar_try_wait(&k_full[s], (g / kStages) & 1) && (g == 0 || mbar_try_wait(s_empty, (g - 1) & 1))) {
-              // S[g] = Q K^T: Q dims 0..383 from tensor memory, 384..575 from shared memory
-              fence_proxy_async_smem();
-              tc_fence_after();
-              const uint64_t kd = sw128_desc(smem_u32(k_ring + s * K_BYTES), 16, 1024);
-              constexpr uint64_t kc = K_CHUNK >> 4, qc = Q_CHUNK >> 4;
-              umma_ts<0>(d_s, a_q + 0, kd + 0, idesc_s);
+        for (int j = 0; j < ntiles; ++j) {
+          const int g = gi + j, s = g % kStages;
+          if (!(ok = mbar_wait(&k_full[s], (g / kStages) & 1, p.err, abort_flag))) break;
+          if (g >= 1 && !(ok = mbar_wait(s_empty, (g - 1) & 1, p.err, abort_flag))) break;
+          // S[g] = Q K^T: Q dims 0..383 from tensor memory, 384..575 from shared memory
+          fence_proxy_async_smem();
+          tc_fence_after();
+          const uint64_t kd = sw128_desc(smem_u32(k_ring + s * K_BYTES), 16, 1024);
+          constexpr uint64_t kc = K_CHUNK >> 4, qc = Q_CHUNK >> 4;
+          umma_ts<0>(d_s, a_q + 0, kd + 0, idesc_s);
 #pragma unroll
-              for (int i = 1; i < 4 * kTmemQChunks; ++i)  // chunk i/4, K step i%4: 8 TMEM columns, 32 B
-                umma_ts<1>(d_s, a_q + (uint32_t)(i * 8), kd + (uint64_t)(i >> 2) * kc + (uint64_t)(i & 3) * 2, idesc_s);
+          for (int i = 1; i < 4 * kTmemQChunks; ++i)  // chunk i/4, K step i%4: 8 TMEM columns, 32 B
+            umma_ts<1>(d_s, a_q + (uint32_t)(i * 8), kd + (uint64_t)(i >> 2) * kc + (uint64_t)(i & 3) * 2, idesc_s);
 #pragma unroll
-              for (int i = 0; i < 4 * (kChunks - kTmemQChunks); ++i)
-                umma_ss<1>(d_s, qd + (uint64_t)(i >> 2) * qc + (uint64_t)(i & 3) * 2,
-                           kd + (uint64_t)(kTmemQChunks + (i >> 2)) * kc + (uint64_t)(i & 3) * 2, idesc_s);
-              mma_commit(s_full);
-              if (ns == ntiles - 1) mma_commit(q_empty);  // last use of Q by this unit
-              ++ns;
-              did = true;
-            }
-          }
-          if (did) {
-            last = clock64();
-          } else if (*abort_flag) {
-            ok = false;
-            break;
-          } else if (clock64() - last > kWaitCycles) {
-            raise_error(p.err, DSA_DEVERR_TIMEOUT);
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
+          for (int i = 0; i < 4 * (kChunks - kTmemQChunks); ++i)
+            umma_ss<1>(d_s, qd + (uint64_t)(i >> 2) * qc + (uint64_t)(i & 3) * 2,
+                       kd + (uint64_t)(kTmemQChunks + (i >> 2)) * kc + (uint64_t)(i & 3) * 2, idesc_s);
+          mma_commit(s_full);
+          if (j == ntiles - 1) mma_commit(q_empty);  // last use of Q by this unit
         }
         gi += ntiles;
       }
@@ -369,7 +340,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(mma_fin);
       mbar_wait(mma_fin, 0, p.err, nullptr);
     }
-  } else {
+  } else if (warp == kPvWarp) {
+    // ------------------------------------------------------------------ P V issuer
+    if (lane == 0) {
+      const uint32_t idesc_o = idesc_f16(1u, 1u, 128u, (uint32_t)kHalf);  // O: B (V) MN-major
+      // P [128 x 64] K-major, no swizzle: 8x16-byte core matrices 128 B apart along K and 1024 B
+      // apart along M; one K step (16 keys) is two core matrices = 256 bytes
+      const uint64_t pd = noswz_desc(smem_u32(p_s), 128, 1024);
+      const uint32_t d_o = tmem + TM_O;
+      int gi = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int t, sp, v;
+        unit_coords(p, u, t, sp, v);
+        const int ntiles = unit_tiles(p, sp);
+        for (int j = 0; j < ntiles; ++j) {
+          const int g = gi + j, s = g % kStages;
+          if (!(ok = mbar_wait(p_full, g & 1, p.err, abort_flag))) break;
+          // O_v += P V_v; V is MN-major 128B-swizzled: 64-dim blocks K_CHUNK apart, 8-row groups
+          // 1024 B apart, one K step (16 rows) = 2048 bytes
+          tc_fence_after();
+          const uint64_t vd = sw128_desc(smem_u32(k_ring + s * K_BYTES) + (uint32_t)(v * 4 * K_CHUNK), K_CHUNK, 1024);
+          if (j > 0)
+            umma_ss<1>(d_o, pd, vd, idesc_o);
+          else
+            umma_ss<0>(d_o, pd, vd, idesc_o);
+          umma_ss<1>(d_o, pd + 16, vd + 128, idesc_o);
+          umma_ss<1>(d_o, pd + 32, vd + 256, idesc_o);
+          umma_ss<1>(d_o, pd + 48, vd + 384, idesc_o);
+          mma_commit(pv_done);
+          mma_commit(&k_empty[s]);
+        }
+        gi += ntiles;
+      }
+      mma_commit(mma_fin);
+      mbar_wait(mma_fin, 0, p.err, nullptr);
+    }
+  } else if (warp < kPvWarp) {
     // ------------------------------------------------------------------ softmax + epilogue
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // head row
@@ -638,8 +645,12 @@ size_t mla_tc_workspace_bytes(int T, int H, int d_v, int nsplit) {
 
 cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_t s) {
   const int T = a.batch.num_queries;
-  alignas(64) CUtensorMap qmap;
+  alignas(64) CUtensorMap qmap, lmap;
   if (!encode_tmap_2d(&qmap, a.q, 2, kDqk, (uint64_t)T * kH, kDqk * 2, 64, kH, true)) return cudaErrorInvalidValue;
+  const uint64_t pool_rows = (uint64_t)a.latent.num_blocks * kPage;
+  if (pool_rows >= 0x7FFFFFFFull) return cudaErrorInvalidValue;  // row coordinates are 32-bit
+  if (!encode_tmap_2d(&lmap, a.latent.data, 2, kDqk, pool_rows, (uint64_t)kDqk * 2, 64, 1, true))
+    return cudaErrorInvalidValue;
   Params p;
   p.latent = static_cast<const __nv_bfloat16*>(a.latent.data);
   p.q = static_cast<const __nv_bfloat16*>(a.q);
@@ -650,6 +661,7 @@ cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.lse = a.lse;
   p.num_blocks = a.latent.num_blocks;
+  p.oob_row = (int32_t)pool_rows;
   p.T = T;
   p.k = a.k;
   p.nsplit = nsplit;
@@ -670,7 +682,7 @@ cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_
   if (e != cudaSuccess) return e;
   const int units = T * nsplit * 2;
   const int grid = units < num_sms ? units : num_sms;
-  mla_tc_kernel<<<grid, kThreads, SMEM, s>>>(qmap, p);
+  mla_tc_kernel<<<grid, kThreads, SMEM, s>>>(qmap, lmap, p);
   e = cudaGetLastError();
   if (e != cudaSuccess || nsplit == 1) return e;
   mla_combine_kernel<<<dim3(T, kH), 128, 0, s>>>(p.part_o, p.part_lse, nsplit, p.out, a.lse);
