@@ -225,6 +225,22 @@ __device__ __forceinline__ void e4m3x16_to_f16(const uint4& in, uint4& lo, uint4
   e4m3x4_to_f16x4(in.w, hi.z, hi.w);
 }
 
+// (a0, a1) * (b0, b1) + c as one packed f32x2 FMA (round to nearest, per lane).
+__device__ __forceinline__ uint64_t ffma2(float a0, float a1, float b0, float b1, uint64_t c) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 a, b;\n\t"
+      "mov.b64 a, {%1, %2};\n\t"
+      "mov.b64 b, {%3, %4};\n\t"
+      "fma.rn.f32x2 %0, a, b, %5;\n\t}"
+      : "=l"(d)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ void unpack2(uint64_t x, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+}
+
 // bf16 x8 -> f16 x8 in place (16 bytes)
 __device__ __forceinline__ uint4 bf16x8_to_f16(const uint4& in) {
   uint4 out;
@@ -550,19 +566,22 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
         tmem_ld16(tbase + qi * 64 + 48, *reinterpret_cast<uint32_t(*)[16]>(&v[48]));
         tmem_wait_ld();
         const float4* w4 = reinterpret_cast<const float4*>(w_mine + qi * kHeads);
-        float acc[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+        // head pairs in packed f32x2 FMAs, four independent pair accumulators
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int h4 = 0; h4 < 16; ++h4) {
           const float4 wv = w4[h4];
-          float* ac = acc + (h4 & 1) * 4;
-          ac[0] = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * h4 + 0]), 0.0f), ac[0]);
-          ac[1] = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * h4 + 1]), 0.0f), ac[1]);
-          ac[2] = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * h4 + 2]), 0.0f), ac[2]);
-          ac[3] = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * h4 + 3]), 0.0f), ac[3]);
+          uint64_t* ac = acc + (h4 & 1) * 2;
+          ac[0] = ffma2(wv.x, wv.y, fmaxf(__uint_as_float(v[4 * h4 + 0]), 0.0f), fmaxf(__uint_as_float(v[4 * h4 + 1]), 0.0f), ac[0]);
+          ac[1] = ffma2(wv.z, wv.w, fmaxf(__uint_as_float(v[4 * h4 + 2]), 0.0f), fmaxf(__uint_as_float(v[4 * h4 + 3]), 0.0f), ac[1]);
         }
-        const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        float sum = 0.0f;
+        {
+          float lo[4], hi[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) unpack2(acc[e], lo[e], hi[e]);
+          sum = ((lo[0] + hi[0]) + (lo[1] + hi[1])) + ((lo[2] + hi[2]) + (lo[3] + hi[3]));
+        }
         if (present && s < npos[qi]) p.scores[(int64_t)(grp * NQ + q0 + qi) * p.ld + s] = sum * scale;
       }
       tc_fence_before();
