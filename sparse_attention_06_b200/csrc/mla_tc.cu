@@ -557,17 +557,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// grid (T, 128 heads), block 128: merge the split partials of one (query, head) row; each thread
-// owns 4 of the 512 value columns.  The split weights exp(LSE_sp - max) are computed once into
-// shared memory, so the per-split loads of the accumulation loop are independent.
+// grid (T, 128 heads), block 256: merge the split partials of one (query, head) row.  The split
+// weights exp(LSE_sp - max) go to shared memory first; then thread i sums column group i % 128
+// (4 of the 512 value columns) over the splits i / 128, i / 128 + 2, ... with up to 16 loads in
+// flight, and the two halves are added through shared memory.
 constexpr int kMaxSplits = 64;
-__global__ void __launch_bounds__(128) mla_combine_kernel(const float* __restrict__ part_o,
-                                                          const float* __restrict__ part_lse, int nsplit,
-                                                          __nv_bfloat16* __restrict__ out,
-                                                          float* __restrict__ lse_out) {
+constexpr int kCombThreads = 256;
+__global__ void __launch_bounds__(kCombThreads) mla_combine_kernel(const float* __restrict__ part_o,
+                                                                   const float* __restrict__ part_lse, int nsplit,
+                                                                   __nv_bfloat16* __restrict__ out,
+                                                                   float* __restrict__ lse_out) {
   __shared__ float wts[kMaxSplits];
-  __shared__ float s_mx, s_inv, s_lse;
-  const int t = blockIdx.x, h = blockIdx.y, c = threadIdx.x * 4;
+  __shared__ float4 red[kCombThreads / 2];
+  __shared__ float s_inv, s_lse;
+  const int t = blockIdx.x, h = blockIdx.y;
+  const int c4 = threadIdx.x & 127, half = threadIdx.x >> 7;
   const int64_t row0 = (int64_t)t * nsplit * kH + h;  // partial row of split 0; split sp adds sp*kH
   if (threadIdx.x < 32) {
     float mx = -INFINITY;
@@ -588,23 +592,38 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const float* __restric
   }
   __syncthreads();
   float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll 8
-  for (int sp = 0; sp < nsplit; ++sp) {
-    const float wgt = wts[sp];
-    const float4 a = __ldg(reinterpret_cast<const float4*>(part_o + (row0 + (int64_t)sp * kH) * kDv + c));
-    acc.x = fmaf(wgt, a.x, acc.x);
-    acc.y = fmaf(wgt, a.y, acc.y);
-    acc.z = fmaf(wgt, a.z, acc.z);
-    acc.w = fmaf(wgt, a.w, acc.w);
+  const float4* src = reinterpret_cast<const float4*>(part_o + row0 * kDv) + c4;
+  const int64_t step = (int64_t)kH * kDv / 4;  // float4s from one split's row to the next
+  for (int sp0 = half; sp0 < nsplit; sp0 += 32) {
+    float4 a[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {  // every load of the batch in flight before the first use
+      const int sp = sp0 + 2 * e;
+      a[e] = sp < nsplit ? __ldg(src + sp * step) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int sp = sp0 + 2 * e;
+      const float wgt = sp < nsplit ? wts[sp] : 0.0f;
+      acc.x = fmaf(wgt, a[e].x, acc.x);
+      acc.y = fmaf(wgt, a[e].y, acc.y);
+      acc.z = fmaf(wgt, a[e].z, acc.z);
+      acc.w = fmaf(wgt, a[e].w, acc.w);
+    }
   }
-  const float inv = s_inv;
-  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-  const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-  uint2 pk;
-  pk.x = *reinterpret_cast<const uint32_t*>(&lo);
-  pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-  *reinterpret_cast<uint2*>(out + ((int64_t)t * kH + h) * kDv + c) = pk;
-  if (lse_out && threadIdx.x == 0) lse_out[(int64_t)t * kH + h] = s_lse;
+  if (half) red[c4] = acc;
+  __syncthreads();
+  if (!half) {
+    const float4 o = red[c4];
+    const float inv = s_inv;
+    const __nv_bfloat162 lo = __floats2bfloat162_rn((acc.x + o.x) * inv, (acc.y + o.y) * inv);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn((acc.z + o.z) * inv, (acc.w + o.w) * inv);
+    uint2 pk;
+    pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(out + ((int64_t)t * kH + h) * kDv + 4 * c4) = pk;
+    if (lse_out && threadIdx.x == 0) lse_out[(int64_t)t * kH + h] = s_lse;
+  }
 }
 
 int split_size(int k, int nsplit) { return ((k + nsplit - 1) / nsplit + kTile - 1) / kTile * kTile; }
@@ -685,7 +704,7 @@ cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_
   mla_tc_kernel<<<grid, kThreads, SMEM, s>>>(qmap, lmap, p);
   e = cudaGetLastError();
   if (e != cudaSuccess || nsplit == 1) return e;
-  mla_combine_kernel<<<dim3(T, kH), 128, 0, s>>>(p.part_o, p.part_lse, nsplit, p.out, a.lse);
+  mla_combine_kernel<<<dim3(T, kH), kCombThreads, 0, s>>>(p.part_o, p.part_lse, nsplit, p.out, a.lse);
   return cudaGetLastError();
 }
 
