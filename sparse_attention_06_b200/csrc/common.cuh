@@ -109,6 +109,17 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* e
 }
 
 // ---------------------------------------------------------------------------------------------
+// programmatic dependent launch
+// ---------------------------------------------------------------------------------------------
+// A kernel launched with programmatic stream serialization may start while the previous kernel
+// of the stream is still running; it must not touch global memory that kernel may write before
+// griddep_wait() returns (which waits for that kernel's completion and memory flush).
+// griddep_launch_dependents() lets the next kernel of the stream begin launching; it takes effect
+// once every CTA of this grid has called it or exited.  Both are no-ops without the attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------------------------
 // async-proxy fences, TMA, cp.async
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -288,6 +288,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  griddep_launch_dependents();
 
   if (tid == 0) {
     for (int i = 0; i < C::OPS; ++i) {
@@ -321,6 +322,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
     tmem_relinquish();
   }
   __syncthreads();
+  griddep_wait();  // inputs may come from the previous kernel of the stream
   // total tile count of the whole call (every CTA computes the same value)
   {
     unsigned long long part = 0;
@@ -696,8 +698,9 @@ cudaError_t launch_impl(const IndexerArgs& a, int num_sms, cudaStream_t s) {
   auto kern = indexer_tc_kernel<NQ, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<num_sms, C::THREADS, C::SMEM, s>>>(kmap, qmap, p);
-  return cudaGetLastError();
+  cudaLaunchAttribute attrs[2];
+  const cudaLaunchConfig_t cfg = launch_config(dim3(num_sms), dim3(C::THREADS), C::SMEM, s, attrs);
+  return cudaLaunchKernelEx(&cfg, kern, kmap, qmap, p);
 }
 
 }  // namespace

@@ -53,6 +53,31 @@ cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_
 int mla_tc_num_splits(int T, int k, int num_sms);
 size_t mla_tc_workspace_bytes(int T, int H, int d_v, int nsplit);
 
+// Launch configuration with programmatic stream serialization (the kernel may start while the
+// previous kernel of the stream finishes; every kernel here waits for it with griddepcontrol.wait
+// before its first global-memory access) and, when cluster_x > 0, thread-block clusters of
+// cluster_x CTAs.  `attrs` must hold two entries and outlive the launch call.
+inline cudaLaunchConfig_t launch_config(dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                        cudaLaunchAttribute* attrs, unsigned cluster_x = 0) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
+  if (cluster_x > 0) {
+    attrs[1].id = cudaLaunchAttributeClusterDimension;
+    attrs[1].val.clusterDim.x = cluster_x;
+    attrs[1].val.clusterDim.y = 1;
+    attrs[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
+  return cfg;
+}
+
 // detail text returned by dsa_last_error_message() on this host thread
 void set_last_error_message(const char* msg);
 

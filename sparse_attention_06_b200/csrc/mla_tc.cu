@@ -175,6 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int units = p.T * p.nsplit * 2;
+  griddep_launch_dependents();
 
   if (tid == 0) {
     if (blockIdx.x < units) {
@@ -205,6 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // the selection comes from the previous kernel of the stream
 
   if (warp < kGatherWarps) {
     // ------------------------------------------------------------------ Q and row gather
@@ -572,6 +574,8 @@ __global__ void __launch_bounds__(kCombThreads) mla_combine_kernel(const float* 
   __shared__ float s_inv, s_lse;
   const int t = blockIdx.x, h = blockIdx.y;
   const int c4 = threadIdx.x & 127, half = threadIdx.x >> 7;
+  griddep_launch_dependents();
+  griddep_wait();  // the partials come from the kernel before
   const int64_t row0 = (int64_t)t * nsplit * kH + h;  // partial row of split 0; split sp adds sp*kH
   if (threadIdx.x < 32) {
     float mx = -INFINITY;
@@ -701,11 +705,14 @@ cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_
   if (e != cudaSuccess) return e;
   const int units = T * nsplit * 2;
   const int grid = units < num_sms ? units : num_sms;
-  mla_tc_kernel<<<grid, kThreads, SMEM, s>>>(qmap, lmap, p);
-  e = cudaGetLastError();
+  cudaLaunchAttribute attrs[2];
+  const cudaLaunchConfig_t cfg = launch_config(dim3(grid), dim3(kThreads), SMEM, s, attrs);
+  e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, qmap, lmap, p);
   if (e != cudaSuccess || nsplit == 1) return e;
-  mla_combine_kernel<<<dim3(T, kH), kCombThreads, 0, s>>>(p.part_o, p.part_lse, nsplit, p.out, a.lse);
-  return cudaGetLastError();
+  cudaLaunchAttribute cattrs[2];
+  const cudaLaunchConfig_t ccfg = launch_config(dim3(T, kH), dim3(kCombThreads), 0, s, cattrs);
+  return cudaLaunchKernelEx(&ccfg, mla_combine_kernel, (const float*)p.part_o, (const float*)p.part_lse, nsplit, p.out,
+                            a.lse);
 }
 
 }  // namespace dsa

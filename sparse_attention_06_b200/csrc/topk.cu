@@ -365,8 +365,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   extern __shared__ __align__(16) uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31;
+  griddep_launch_dependents();
   const uint32_t C = cluster_nctas(), r = cluster_rank();
   const int64_t t = cluster_index();
+  griddep_wait();  // the scores come from the previous kernel of the stream
   int64_t n = (int64_t)q_pos[t] + 1;
   if (n > ld) {  // a row cannot hold more scores than its stride
     if (tid == 0 && r == 0) raise_error(err, DSA_DEVERR_REQUEST);
@@ -603,18 +605,9 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, i
   const int smem = (int)sizeof(Smem);
   e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((int64_t)T * C), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cudaLaunchAttribute attrs[2];
+  const cudaLaunchConfig_t cfg = launch_config(dim3((unsigned)((int64_t)T * C)), dim3(kThreads), (size_t)smem, s,
+                                               attrs, (unsigned)C);
   return cudaLaunchKernelEx(&cfg, topk_kernel, scores, ld, q_pos, k, idx, err);
 }
 
