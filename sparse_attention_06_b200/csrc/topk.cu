@@ -46,7 +46,7 @@ constexpr int kCap = 6144;                 // candidates of one row (all CTAs of
 constexpr int kMaxSlice = 1 << 17;         // positions one CTA's bitmap covers
 constexpr int kMaxCluster = 8;
 constexpr int kSample = 4096;              // sampled keys (512 chunks of 8)
-constexpr int kPer = 8;                    // scores per thread per filter step
+constexpr int kPer = 16;                   // scores per thread per filter step
 
 struct Smem {
   uint32_t bitmap[kMaxSlice / 32];      // selected positions of this CTA's slice
@@ -359,7 +359,7 @@ __device__ __forceinline__ void load_batch(const float* srow, int len, int base,
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     topk_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ q_pos, int k,
                 int32_t* __restrict__ idx, int* err) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -435,9 +435,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   __syncthreads();
 
-  // 2. filter: append (key, position) of every score >= tau in this slice
+  // 2. filter: append (key, position) of every score >= tau in this slice; the next batch's loads
+  //    are issued before the current batch is processed
   for (int base = 0; base < len; base += kStep) {
-    if (base > 0) load_batch(srow, len, base, vec, v);
+    float vn[kPer];
+    if (base + kStep < len) load_batch(srow, len, base + kStep, vec, vn);
     uint32_t mask = 0u;
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
@@ -466,6 +468,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
     }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) v[j] = vn[j];
   }
   __syncthreads();
   if (tid < (int)C) st_cluster_u32(&S.cnt_all[r], (uint32_t)tid, S.scal[5]);
