@@ -22,8 +22,10 @@
 //               the following batch already in flight), then issues the TMA copies of key pages
 //               and query tiles into 128B-swizzled shared memory and records each tile's block
 //               ids in a tile-info ring
-//   warp 1      TMEM allocation and the single thread that issues tcgen05.mma / tcgen05.commit
-//   epilogue    4 warps (8 when 4 queries share a tile, each warp half of them): reads the tile
+//   warp 1      TMEM allocation and the thread that issues tcgen05.mma / tcgen05.commit (for e4m3
+//               keys with one query per tile, of the even tiles; the last warp issues the odd ones)
+//   epilogue    8 warps in two sets (alternate tiles with one query per tile, else half of the
+//               queries each): reads the tile
 //               info LOOK tiles ahead (and, for e4m3, starts a 4-byte cp.async of its key's scale
 //               then), then per tile: tcgen05.ld of the accumulator, ReLU, head sum, scale, score
 //               stores
@@ -77,7 +79,16 @@ struct Cfg {
   static constexpr int EPI_ARRIVE = EPI_ALT ? 4 : 8;          // epilogue arrivals per tile
   static constexpr int CONV_WARPS = FP8 ? 4 : 0;
   static constexpr int CONV0 = 2 + EPI_WARPS;                 // first converter warp
-  static constexpr int THREADS = 32 * (CONV0 + CONV_WARPS);
+  // One thread issues a tcgen05.mma about every 60 cycles, which at N = 64 is half the tensor
+  // pipe's rate: for e4m3 keys with one query per tile (A in tensor memory) a second warp issues
+  // the odd tiles (accumulator 1).
+  static constexpr int MMA_WARPS = TMEM_A ? 2 : 1;
+  static constexpr int MMA2 = CONV0 + CONV_WARPS;             // the second issuing warp
+  static constexpr int THREADS = 32 * (CONV0 + CONV_WARPS + MMA_WARPS - 1);
+  // Each issuer waits on an operand stage's mbarrier by phase parity, which is only sound when it
+  // has seen the stage's previous phase: with two issuers alternating tiles, every stage must
+  // belong to one of them (an even number of stages).
+  static_assert(MMA_WARPS == 1 || OPS % 2 == 0, "operand stages must not alternate between issuers");
   // shared-memory carve-up (offsets from a 1024-aligned base)
   static constexpr int OFF_OP = 0;
   static constexpr int OFF_ST = OFF_OP + (TMEM_A ? 0 : OPS * OP_BYTES);
@@ -301,14 +312,14 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
     }
     for (int i = 0; i < C::QS; ++i) {
       mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 1);
+      mbar_init(&q_empty[i], C::MMA_WARPS);
       mbar_init(&q_ready[i], C::CONV_WARPS);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], C::EPI_ARRIVE);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, C::MMA_WARPS);
     for (int i = 0; i < C::TIS; ++i) {
       mbar_init(&ti_full[i], 1);
       mbar_init(&ti_empty[i], C::EPI_ARRIVE);
@@ -441,8 +452,9 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
           if (m >= q) drain_wait(&q_full[q], (uint32_t)(((m - q) / C::QS) & 1), p.err);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || (C::MMA_WARPS == 2 && warp == C::MMA2)) {
+    // ------------------------------------------------------------------ MMA issuer(s)
+    const int par = warp == 1 ? 0 : 1;  // with two issuers: the parity of the tiles this one issues
     if (lane == 0 && lo < hi) {
       const uint32_t idesc = idesc_f16(FP8 ? 0u : 1u, 0u, 128u, (uint32_t)C::N);  // f16 or bf16
       Walk<NQ> W;
@@ -457,6 +469,10 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
           ++m;
           slot = m % C::QS;
           if (!(ok = mbar_wait(FP8 ? &q_ready[slot] : &q_full[slot], (m / C::QS) & 1, p.err, abort_flag))) break;
+        }
+        if (C::MMA_WARPS == 2 && (int)(i & 1) != par) {  // the other issuer's tile
+          ++i;
+          continue;
         }
         const int s = (int)(i % C::OPS), use = (int)(i / C::OPS);
         if (!(ok = mbar_wait(&op_full[s], use & 1, p.err, abort_flag))) break;
