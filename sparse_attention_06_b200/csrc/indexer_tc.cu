@@ -413,7 +413,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
               last = grp;
             }
             {
-              if (FP8) {
+              if constexpr (FP8) {
                 const int s = (int)(i % C::STS), use = (int)(i / C::STS);
                 if (use >= 1 && !(ok = mbar_wait(&st_empty[s], (use - 1) & 1, p.err, abort_flag))) goto issued;
                 mbar_arrive_expect_tx(&st_full[s], (b0 >= 0 ? 8192u : 0u) + (b1 >= 0 ? 8192u : 0u));
@@ -446,8 +446,10 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
         // give up: let the copies already issued land before the CTA's memory goes away
         for (int s = 0; s < C::OPS && !FP8; ++s)
           if (i > s) drain_wait(&op_full[s], (uint32_t)(((i - 1 - s) / C::OPS) & 1), p.err);
-        for (int s = 0; s < C::STS; ++s)
-          if (i > s) drain_wait(&st_full[s], (uint32_t)(((i - 1 - s) / C::STS) & 1), p.err);
+        if constexpr (FP8) {
+          for (int s = 0; s < C::STS; ++s)
+            if (i > s) drain_wait(&st_full[s], (uint32_t)(((i - 1 - s) / C::STS) & 1), p.err);
+        }
         for (int q = 0; q < C::QS; ++q)
           if (m >= q) drain_wait(&q_full[q], (uint32_t)(((m - q) / C::QS) & 1), p.err);
       }
@@ -484,7 +486,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
         const uint64_t bd = sw128_desc(smem_u32(q_slots + slot * C::Q_BYTES), 16, 1024);
         const uint32_t d = tmem_base + (uint32_t)(a * C::N);
         constexpr uint64_t ac = C::CHUNK_BYTES >> 4, bc = C::Q_CHUNK >> 4;
-        if (C::TMEM_A) {
+        if constexpr (C::TMEM_A) {
           // A = the f16 key tile in tensor memory: one K step of 16 dims = 8 columns
           const uint32_t at = tmem_base + (uint32_t)(C::A_COL0 + s * C::A_COLS);
           umma_ts<0>(d, at, bd, idesc);
@@ -609,7 +611,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
       ++i;
     }
     cp_async_wait_all();  // no copy may land after the CTA's shared memory is released
-  } else if (FP8) {
+  } else if constexpr (FP8) {
     // ------------------------------------------------------------------ fp8 -> f16 converter
     const int cw = warp - C::CONV0;  // 0 .. CONV_WARPS-1
     const int ct = tid - 32 * C::CONV0;
@@ -636,7 +638,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
       const int so = (int)(i % C::OPS), uo = (int)(i / C::OPS);
       if (uo >= 1 && !warp_wait(&op_empty[so], (uo - 1) & 1, p.err, abort_flag)) break;
       const uint8_t* src = st_ring + s8 * C::ST_BYTES;
-      if (C::TMEM_A) {
+      if constexpr (C::TMEM_A) {
         // this thread: key row `row` (its TMEM lane); the staging tile is 128B-swizzled, so the
         // lanes of a warp read distinct banks
         tc_fence_after();

@@ -100,10 +100,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 // Unit u -> (t, split, half): the two halves of one (t, split) are adjacent so that they run
 // concurrently and the second gather of each row hits L2.
 __device__ __forceinline__ void unit_coords(const Params& p, int u, int& t, int& sp, int& v) {
