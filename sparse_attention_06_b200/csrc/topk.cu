@@ -31,6 +31,11 @@
 // Exact path: a radix select over the row finds Tk and the number of ties to take, and an
 // in-order pass over 8192-score chunks writes the positions.
 // Every count is order-independent, so the result does not depend on the order of atomics.
+//
+// Code size.  With few rows the kernel is one serial chain of short phases, each run once per
+// launch, so fetching instructions is a large part of its time.  The radix selection is therefore
+// one out-of-line function over keys in shared memory, shared by the sample, the candidates and
+// the ties; reductions use redux.sync; the exact fallback path is out of line as well.
 #include "common.cuh"
 #include "internal.h"
 
@@ -47,23 +52,27 @@ constexpr int kMaxSlice = 1 << 17;         // positions one CTA's bitmap covers
 constexpr int kMaxCluster = 8;
 constexpr int kSample = 4096;              // sampled keys (512 chunks of 8)
 constexpr int kPer = 16;                   // scores per thread per filter step
+static_assert(kHBins == 8 * kThreads, "each thread scans 8 histogram bins");
+static_assert(kCap >= kSample, "the sample fits the key pool");
 
 struct Smem {
   uint32_t bitmap[kMaxSlice / 32];      // selected positions of this CTA's slice
   uint32_t cand_key[kCap];              // this CTA's candidates (read by the whole cluster)
   uint32_t cand_pos[kCap];
-  uint32_t pool[kCap];                  // the row's candidate keys, then this CTA's ties
-  uint32_t hist[2][kHBins];             // radix histograms, alternating between steps
+  uint32_t pool[kCap];                  // sample keys, then the row's candidate keys, then this CTA's ties
+  alignas(16) uint32_t hist[2][kHBins]; // radix histograms, alternating between steps
   uint32_t red[2 * kWarps];
   uint32_t wsum[kWarps];
-  uint32_t warp_tot[kWarps + 1];
+  uint32_t warp_tot[kWarps];
   uint32_t res[2][4];                   // digit, keys above it, keys in it
   uint32_t scal[12];
   uint32_t cnt_all[kMaxCluster];        // written by every CTA of the cluster: its candidates
   uint32_t above_all[kMaxCluster];      // ... its keys above Tk
   uint32_t ties_all[kMaxCluster];       // ... its keys equal to Tk
 };
-static_assert(kCap >= kSample, "the sample fits the candidate key buffer");
+
+extern __shared__ __align__(16) uint8_t topk_smem[];
+__device__ __forceinline__ Smem& smem() { return *reinterpret_cast<Smem*>(topk_smem); }
 
 // ---------------------------------------------------------------------------------------------
 // cluster primitives (thread-block clusters, distributed shared memory)
@@ -89,6 +98,10 @@ __device__ __forceinline__ uint32_t cluster_index() {
 // Every thread of every CTA of the cluster arrives (release) / waits (acquire).
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+// Arrive without release semantics: only for an arrive that publishes no memory operation.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_sync() {
   cluster_arrive();
   cluster_wait();
@@ -144,104 +157,132 @@ __device__ __forceinline__ uint32_t warp_inclusive_scan(uint32_t v) {
 }
 
 // Exclusive prefix sum of `v` over the block; returns the prefix, writes the block total.
-__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_tot, uint32_t& total) {
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t& total) {
+  Smem& S = smem();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t incl = warp_inclusive_scan(v);
-  if (lane == 31) warp_tot[warp] = incl;
+  if (lane == 31) S.warp_tot[warp] = incl;
   __syncthreads();
-  uint32_t before = 0u, all = 0u;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    const uint32_t x = warp_tot[w];
-    before += w < warp ? x : 0u;
-    all += x;
-  }
-  total = all;
+  const uint32_t x = lane < kWarps ? S.warp_tot[lane] : 0u;
+  total = __reduce_add_sync(0xFFFFFFFFu, x);
+  const uint32_t before = __reduce_add_sync(0xFFFFFFFFu, lane < warp ? x : 0u);
   __syncthreads();  // warp_tot is reused by the next scan
   return before + incl - v;
 }
 
-// Clears both radix histograms (each thread its share).  Call before the first kth_key of a CTA;
-// kth_key leaves them clear again.
-__device__ __forceinline__ void clear_hists(Smem& S) {
-  constexpr int kPerT = kHBins / kThreads;
-#pragma unroll
-  for (int b = 0; b < kPerT; ++b) {
-    S.hist[0][threadIdx.x * kPerT + b] = 0u;
-    S.hist[1][threadIdx.x * kPerT + b] = 0u;
-  }
+// Clears both radix histograms (each thread its 8 bins of each).  Call before the first kth_key
+// of a CTA; kth_key leaves them clear again.
+__device__ __forceinline__ void clear_hist(int which) {
+  uint4* h = reinterpret_cast<uint4*>(smem().hist[which]) + 2 * threadIdx.x;
+  h[0] = make_uint4(0u, 0u, 0u, 0u);
+  h[1] = make_uint4(0u, 0u, 0u, 0u);
 }
 
-// j-th largest (1-based) of the keys that each(f) hands to f, over the block, by radix steps of
+// Keys held in registers: element e of this thread is key tid + e * kThreads, valid below m.
+struct RegKeys {
+  static constexpr int N = kCap / kThreads;
+  uint32_t v[N];
+  int m;
+  template <class F>
+  __device__ __forceinline__ void operator()(F f) const {
+#pragma unroll
+    for (int e = 0; e < N; ++e)
+      if ((int)threadIdx.x + e * kThreads < m) f(v[e]);
+  }
+};
+
+// Keys in shared memory: the first m entries of the pool, or of this CTA's candidate keys.  They
+// are loaded into registers once per selection (load()), so that the histogram passes issue
+// their atomics back to back.
+struct SmemKeys {
+  int m;
+  bool cand;
+  __device__ __forceinline__ RegKeys load() const {
+    const uint32_t* keys = cand ? smem().cand_key : smem().pool;
+    RegKeys r;
+    r.m = m;
+#pragma unroll
+    for (int e = 0; e < RegKeys::N; ++e) {
+      const int i = threadIdx.x + e * kThreads;
+      r.v[e] = i < m ? keys[i] : 0u;
+    }
+    return r;
+  }
+};
+
+// The keys of a whole row in global memory (exact path); a NaN score sets the CTA's NaN flag.
+struct RowKeys {
+  const float* row;
+  int64_t n;
+  __device__ __forceinline__ RowKeys load() const { return *this; }
+  template <class F>
+  __device__ __forceinline__ void operator()(F f) const {
+    bool nan = false;
+    for (int64_t i = threadIdx.x; i < n; i += kThreads) f(order_key(row[i], nan));
+    if (nan) smem().scal[4] = 1u;  // benign race: every writer stores 1
+  }
+};
+
+struct Kth {
+  uint32_t key;    // the selected key (exact) or the threshold (not exact)
+  uint32_t above;  // exact: keys strictly greater than `key`
+};
+
+// j-th largest (1-based) of the keys that src(f) hands to f, over the block, by radix steps of
 // 12-bit digits taken from the highest bit in which the keys differ (bits every key shares are
 // skipped).  After each step only the keys in the chosen digit bin stay in play.
-//   exact:  returns that key; *above = the number of keys strictly greater.
+//   exact:  returns that key and the number of keys strictly greater.
 //   !exact: stops after the first step whose chosen bin holds at most `limit` keys and returns the
 //           bin's lower edge (the undecided low bits zero): at least j keys are >= the result.
 // j must not exceed the number of keys.  Three block barriers per step (histogram, warp sums,
 // result); the histograms alternate between steps, so clearing one overlaps the other's use.
-template <class Each>
-__device__ uint32_t kth_key(Smem& S, uint32_t j, Each each, bool exact, uint32_t limit, uint32_t* above) {
+template <class Src>
+__device__ __noinline__ Kth kth_key(Src keys, uint32_t j, bool exact, uint32_t limit) {
+  Smem& S = smem();
+  const auto src = keys.load();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t a = 0xFFFFFFFFu, o = 0u;
-  each([&](uint32_t key) {
+  src([&](uint32_t key) {
     a &= key;
     o |= key;
   });
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    a &= __shfl_xor_sync(0xFFFFFFFFu, a, off);
-    o |= __shfl_xor_sync(0xFFFFFFFFu, o, off);
-  }
+  a = __reduce_and_sync(0xFFFFFFFFu, a);
+  o = __reduce_or_sync(0xFFFFFFFFu, o);
   if (lane == 0) {
     S.red[warp] = a;
     S.red[kWarps + warp] = o;
   }
   __syncthreads();
-  a = 0xFFFFFFFFu;
-  o = 0u;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    a &= S.red[w];
-    o |= S.red[kWarps + w];
-  }
+  a = __reduce_and_sync(0xFFFFFFFFu, lane < kWarps ? S.red[lane] : 0xFFFFFFFFu);
+  o = __reduce_or_sync(0xFFFFFFFFu, lane < kWarps ? S.red[kWarps + lane] : 0u);
   uint32_t fixed = ~(a ^ o);  // decided bits: those every key shares, then each chosen digit
   uint32_t prefix = a & fixed;
   uint32_t krem = j;
   int buf = 0;
-  constexpr int kPerLane = kHBins / kThreads;  // bins per thread (8)
-  constexpr int kPerWarp = kHBins / kWarps;    // bins per warp (256)
   while (fixed != 0xFFFFFFFFu) {
     const int hb = 31 - __clz(~fixed);
     const int lb = hb >= kDigit - 1 ? hb - (kDigit - 1) : 0;
     const uint32_t dmask = (2u << (hb - lb)) - 1u;
     uint32_t* hist = S.hist[buf];
-    each([&](uint32_t key) {
+    src([&](uint32_t key) {
       if ((key & fixed) == prefix) atomicAdd(&hist[(key >> lb) & dmask], 1u);
     });
-#pragma unroll
-    for (int b = 0; b < kPerLane; ++b) S.hist[buf ^ 1][tid * kPerLane + b] = 0u;
+    clear_hist(buf ^ 1);
     __syncthreads();
-    // warp w owns bins [kHBins - kPerWarp (w + 1), kHBins - kPerWarp w), lane l the kPerLane bins
-    // below kHBins - kPerWarp w - kPerLane l: counts run downward from the top bin
-    uint32_t h[kPerLane];
-    uint32_t lsum = 0u;
-    const int top = kHBins - 1 - warp * kPerWarp - lane * kPerLane;
-#pragma unroll
-    for (int b = 0; b < kPerLane; ++b) {
-      h[b] = hist[top - b];
-      lsum += h[b];
-    }
+    // thread tid owns the 8 bins [8 (kThreads - 1 - tid), 8 (kThreads - tid)); counts run downward
+    // from the top bin (thread 0) to bin 0 (the last thread)
+    const uint4* mine = reinterpret_cast<const uint4*>(hist) + 2 * (kThreads - 1 - tid);
+    const uint4 lo4 = mine[0], hi4 = mine[1];
+    const uint32_t h[8] = {hi4.w, hi4.z, hi4.y, hi4.x, lo4.w, lo4.z, lo4.y, lo4.x};
+    const uint32_t lsum = (lo4.x + lo4.y) + (lo4.z + lo4.w) + (hi4.x + hi4.y) + (hi4.z + hi4.w);
     const uint32_t lincl = warp_inclusive_scan(lsum);
     if (lane == 31) S.wsum[warp] = lincl;
     __syncthreads();
-    uint32_t wabove = 0u;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) wabove += w < warp ? S.wsum[w] : 0u;
-    uint32_t abv = wabove + lincl - lsum;
+    uint32_t abv = __reduce_add_sync(0xFFFFFFFFu, lane < warp ? S.wsum[lane] : 0u) + lincl - lsum;
     if (abv < krem && krem <= abv + lsum) {
+      const int top = kHBins - 1 - 8 * tid;
 #pragma unroll
-      for (int b = 0; b < kPerLane; ++b) {
+      for (int b = 0; b < 8; ++b) {
         if (abv < krem && krem <= abv + h[b]) {
           S.res[buf][0] = (uint32_t)(top - b);
           S.res[buf][1] = abv;
@@ -260,50 +301,19 @@ __device__ uint32_t kth_key(Smem& S, uint32_t j, Each each, bool exact, uint32_t
   }
   // the histogram of the last step is the dirty one: clear it for the next call (the next call
   // writes it only after a barrier that follows this)
-#pragma unroll
-  for (int b = 0; b < kPerLane; ++b) S.hist[buf ^ 1][tid * kPerLane + b] = 0u;
-  if (above) *above = j - krem;
-  return prefix & fixed;
-}
-
-// Keys held in registers: element e of this thread is valid when tid + e * kThreads < m.
-template <int N>
-struct RegKeys {
-  uint32_t v[N];
-  int m;
-  template <class F>
-  __device__ __forceinline__ void operator()(F f) const {
-#pragma unroll
-    for (int e = 0; e < N; ++e)
-      if ((int)threadIdx.x + e * kThreads < m) f(v[e]);
-  }
-};
-
-template <int N>
-__device__ __forceinline__ RegKeys<N> load_keys(const uint32_t* src, int m, bool complement) {
-  RegKeys<N> r;
-  r.m = m;
-#pragma unroll
-  for (int e = 0; e < N; ++e) {
-    const int i = threadIdx.x + e * kThreads;
-    const uint32_t x = i < m ? src[i] : 0u;
-    r.v[e] = complement ? ~x : x;
-  }
-  return r;
+  clear_hist(buf ^ 1);
+  return Kth{prefix & fixed, j - krem};
 }
 
 // Exact path over a whole row in global memory: radix select of Tk, then an in-order pass over
 // chunks of kPer * kThreads scores (each thread takes kPer consecutive positions) with two
 // block-wide prefix sums per chunk, one over ties and one over the positions taken.
-__device__ void topk_exact(Smem& S, const float* row, int64_t n, int k, int32_t* out, bool& saw_nan) {
-  clear_hists(S);
+__device__ __noinline__ void topk_exact(const float* row, int64_t n, int k, int32_t* out) {
+  clear_hist(0);
+  clear_hist(1);
   __syncthreads();
-  uint32_t above;
-  auto each = [&](auto f) {
-    for (int64_t i = threadIdx.x; i < n; i += kThreads) f(order_key(row[i], saw_nan));
-  };
-  const uint32_t tk = kth_key(S, (uint32_t)k, each, true, 0u, &above);
-  const uint32_t need = (uint32_t)k - above;  // keys equal to tk to take, lowest positions first
+  const Kth tk = kth_key(RowKeys{row, n}, (uint32_t)k, true, 0u);
+  const uint32_t need = (uint32_t)k - tk.above;  // keys equal to Tk to take, lowest positions first
   uint32_t base = 0u, eq_seen = 0u;
   for (int64_t c0 = 0; c0 < n; c0 += (int64_t)kPer * kThreads) {
     const int64_t p0 = c0 + (int64_t)threadIdx.x * kPer;
@@ -313,33 +323,40 @@ __device__ void topk_exact(Smem& S, const float* row, int64_t n, int k, int32_t*
     for (int e = 0; e < kPer; ++e) {
       bool dummy = false;
       key[e] = p0 + e < n ? order_key(row[p0 + e], dummy) : 0u;
-      eq += (p0 + e < n && key[e] == tk) ? 1u : 0u;
+      eq += (p0 + e < n && key[e] == tk.key) ? 1u : 0u;
     }
     uint32_t eq_tot, take_tot;
-    uint32_t eq_rank = eq_seen + block_exclusive_scan(eq, S.warp_tot, eq_tot);
+    uint32_t eq_rank = eq_seen + block_exclusive_scan(eq, eq_tot);
     uint32_t mask = 0u;
 #pragma unroll
     for (int e = 0; e < kPer; ++e) {
       if (p0 + e < n) {
-        if (key[e] > tk) {
+        if (key[e] > tk.key) {
           mask |= 1u << e;
-        } else if (key[e] == tk) {
+        } else if (key[e] == tk.key) {
           if (eq_rank < need) mask |= 1u << e;
           ++eq_rank;
         }
       }
     }
-    uint32_t at = base + block_exclusive_scan((uint32_t)__popc(mask), S.warp_tot, take_tot);
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) {
-      if (mask & (1u << e)) {
-        if (at < (uint32_t)k) out[at] = (int32_t)(p0 + e);
-        ++at;
-      }
+    uint32_t at = base + block_exclusive_scan((uint32_t)__popc(mask), take_tot);
+    while (mask) {
+      const int e = __ffs(mask) - 1;
+      mask &= mask - 1u;
+      if (at < (uint32_t)k) out[at] = (int32_t)(p0 + e);
+      ++at;
     }
     base += take_tot;
     eq_seen += eq_tot;
   }
+}
+
+// v[j] for a j known only at run time, without indexing the register array
+__device__ __forceinline__ float pick(const float (&v)[kPer], int j) {
+  float x = v[0];
+#pragma unroll
+  for (int e = 1; e < kPer; ++e) x = j == e ? v[e] : x;
+  return x;
 }
 
 // kPer scores of a slice for this thread, from 16-byte loads where the slice allows: element
@@ -362,12 +379,14 @@ __device__ __forceinline__ void load_batch(const float* srow, int len, int base,
 __global__ void __launch_bounds__(kThreads, 1)
     topk_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ q_pos, int k,
                 int32_t* __restrict__ idx, int* err) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  Smem& S = *reinterpret_cast<Smem*>(smem_raw);
+  Smem& S = smem();
   const int tid = threadIdx.x, lane = tid & 31;
   griddep_launch_dependents();
   const uint32_t C = cluster_nctas(), r = cluster_rank();
   const int64_t t = cluster_index();
+  // warm the address translation of this row (a prefetch reads nothing that the previous kernel
+  // may still write: the loads below come after the wait)
+  if (tid == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(scores + t * ld + min((int64_t)r * 4096, ld - 1)));
   griddep_wait();  // the scores come from the previous kernel of the stream
   int64_t n = (int64_t)q_pos[t] + 1;
   if (n > ld) {  // a row cannot hold more scores than its stride
@@ -380,21 +399,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   const float* row = scores + t * ld;
-  bool saw_nan = false;
   if (tid == 0) S.scal[4] = 0u;  // NaN seen
-  const int64_t per = (((n + C - 1) / C) + 31) & ~int64_t(31);
-  if (per > kMaxSlice) {  // slices too long for the bitmap: exact path on one CTA
+  if (n > (int64_t)kMaxSlice * C) {  // slices too long for the bitmap: exact path on one CTA
     if (r == 0) {
-      topk_exact(S, row, n, k, out, saw_nan);
-      if (saw_nan) S.scal[4] = 1u;
+      __syncthreads();  // the NaN flag is clear
+      topk_exact(row, n, k, out);
       __syncthreads();
       if (tid == 0 && S.scal[4]) raise_error(err, DSA_DEVERR_NAN_SCORE);
     }
     return;
   }
-  const int64_t lo = min(n, (int64_t)r * per);
-  const int64_t hi = min(n, lo + per);
-  const int len = (int)(hi - lo);
+  // slices of a multiple of 32 positions (whole bitmap words), at most kMaxSlice; n < 2^20 here
+  const int nn = (int)n;
+  const int per = (int)((((uint32_t)nn + C - 1u) / C + 31u) & ~31u);
+  const int lo = min(nn, (int)r * per);
+  const int len = min(nn, lo + per) - lo;
   const int words = (len + 31) >> 5;
   const float* srow = row + lo;
   const bool vec = ((reinterpret_cast<uintptr_t>(srow) & 15u) == 0);
@@ -402,12 +421,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   float v[kPer];
   load_batch(srow, len, 0, vec, v);  // the first batch of this slice, in flight during step 1
   for (int w = tid; w < words; w += kThreads) S.bitmap[w] = 0u;
-  clear_hists(S);
+  clear_hist(0);
+  clear_hist(1);
   if (tid == 0) {
     S.scal[5] = 0u;  // candidates of this CTA
     S.scal[6] = 0u;  // ties of this CTA
     S.scal[7] = 0u;  // keys above Tk in this CTA
   }
+  bool saw_nan = false;
 
   // 1. threshold from a strided sample (identical in every CTA of the cluster)
   const bool take_all = n <= kCap;
@@ -415,8 +436,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (!take_all) {
     constexpr int kChunks = kSample / 8;
     constexpr int kSPT = kSample / kThreads;
-    RegKeys<kSPT> smp;
-    smp.m = kSample;
     float sv[kSPT];
 #pragma unroll
     for (int e = 0; e < kSPT; ++e) {
@@ -424,16 +443,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t p = (((int64_t)(s >> 3) * n / kChunks) & ~int64_t(7)) + (s & 7);
       sv[e] = row[p];
     }
+    // the first batch is consumed here (NaN check), so that its loads complete with the sample's
+    // rather than after step 1
 #pragma unroll
-    for (int e = 0; e < kSPT; ++e) smp.v[e] = order_key(sv[e], saw_nan);
-    __syncthreads();  // histograms cleared
+    for (int j = 0; j < kPer; ++j) saw_nan |= v[j] != v[j];
+#pragma unroll
+    for (int e = 0; e < kSPT; ++e) S.pool[tid + e * kThreads] = order_key(sv[e], saw_nan);
+    __syncthreads();  // sample keys and cleared histograms visible
     const float rk = (float)k * (float)kSample / (float)n;  // sample rank of the row's K-th score
     int js = (int)ceilf(1.15f * rk + 4.f * sqrtf(rk) + 8.f);
     js = min(js, kSample);
-    const uint32_t tau = kth_key(S, (uint32_t)js, smp, false, (uint32_t)(js / 8 + 2), nullptr);
-    tau_f = key_to_float(tau);
+    tau_f = key_to_float(kth_key(SmemKeys{kSample, false}, (uint32_t)js, false, (uint32_t)(js / 8 + 2)).key);
+  } else {
+    __syncthreads();  // the counters are clear
   }
-  __syncthreads();
 
   // 2. filter: append (key, position) of every score >= tau in this slice; the next batch's loads
   //    are issued before the current batch is processed
@@ -456,68 +479,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t wbase = 0u;
       if (lane == 0) wbase = atomicAdd(&S.scal[5], tot);
       uint32_t at = __shfl_sync(0xFFFFFFFFu, wbase, 0) + incl - c;
-#pragma unroll
-      for (int j = 0; j < kPer; ++j) {
-        if (mask & (1u << j)) {
-          if (at < (uint32_t)kCap) {
-            bool dummy = false;
-            S.cand_key[at] = order_key(v[j], dummy);
-            S.cand_pos[at] = (uint32_t)(lo + base + ((j >> 2) * kThreads + tid) * 4 + (j & 3));
-          }
-          ++at;
-        }
+      for (uint32_t mm = mask; mm != 0u && at < (uint32_t)kCap; mm &= mm - 1u, ++at) {
+        const int j = __ffs(mm) - 1;
+        bool dummy = false;
+        S.cand_key[at] = order_key(pick(v, j), dummy);
+        S.cand_pos[at] = (uint32_t)(lo + base + ((j >> 2) * kThreads + tid) * 4 + (j & 3));
       }
     }
 #pragma unroll
     for (int j = 0; j < kPer; ++j) v[j] = vn[j];
   }
+  if (saw_nan) S.scal[4] = 1u;  // benign race: every writer stores 1
   __syncthreads();
   if (tid < (int)C) st_cluster_u32(&S.cnt_all[r], (uint32_t)tid, S.scal[5]);
   cluster_sync();  // A: every CTA's candidates and counts are visible to the cluster
 
   uint32_t m = 0u;  // the row's candidates
-#pragma unroll
-  for (int q = 0; q < kMaxCluster; ++q) m += q < (int)C ? S.cnt_all[q] : 0u;
+  for (int q = 0; q < (int)C; ++q) m += S.cnt_all[q];
   if (m < (uint32_t)k || m > (uint32_t)kCap) {
     // the threshold missed (too high, or too many scores tie at it): exact path on CTA 0
     cluster_sync();  // no CTA reads another's shared memory after this point
-    if (r == 0) topk_exact(S, row, n, k, out, saw_nan);
-    if (saw_nan) S.scal[4] = 1u;
-    __syncthreads();
-    if (tid == 0 && S.scal[4]) raise_error(err, DSA_DEVERR_NAN_SCORE);
+    if (r == 0) {
+      topk_exact(row, n, k, out);
+      __syncthreads();
+      if (tid == 0 && S.scal[4]) raise_error(err, DSA_DEVERR_NAN_SCORE);
+    }
     return;
   }
 
-  // 3. exact K-th key among the row's candidates (gathered from every CTA of the cluster)
-  constexpr int kKPT = kCap / kThreads;
-  RegKeys<kKPT> cand;
-  cand.m = (int)m;
+  // 3. exact K-th key among the row's candidates (gathered from every CTA of the cluster into the
+  //    pool, CTA by CTA; the first 512 of each CTA's keys are loaded at once)
   if (C > 1) {
-    uint32_t pre[kMaxCluster];  // candidate offsets of the cluster's CTAs
-    pre[0] = 0u;
+    uint32_t val[kMaxCluster];
 #pragma unroll
-    for (int q = 1; q < kMaxCluster; ++q) pre[q] = pre[q - 1] + (q - 1 < (int)C ? S.cnt_all[q - 1] : 0u);
-#pragma unroll
-    for (int e = 0; e < kKPT; ++e) {
-      const uint32_t i = (uint32_t)(tid + e * kThreads);
-      uint32_t src = 0u, off = 0u;
-#pragma unroll
-      for (int q = 1; q < kMaxCluster; ++q) {
-        if (pre[q] <= i && q < (int)C) {
-          src = (uint32_t)q;
-          off = pre[q];
-        }
-      }
-      cand.v[e] = i < m ? ld_cluster_u32(&S.cand_key[i - off], src) : 0u;
+    for (int q = 0; q < kMaxCluster; ++q) {
+      const uint32_t cq = q < (int)C ? S.cnt_all[q] : 0u;
+      val[q] = (uint32_t)tid < cq ? ld_cluster_u32(&S.cand_key[tid], (uint32_t)q) : 0u;
     }
-  } else {
-    cand = load_keys<kKPT>(S.cand_key, (int)m, false);
+    uint32_t pre = 0u;
+    for (int q = 0; q < (int)C; ++q) {
+      const uint32_t cq = S.cnt_all[q];
+      if ((uint32_t)tid < cq) S.pool[pre + tid] = val[q];
+      for (uint32_t i = tid + kThreads; i < cq; i += kThreads) S.pool[pre + i] = ld_cluster_u32(&S.cand_key[i], (uint32_t)q);
+      pre += cq;
+    }
+    __syncthreads();
   }
-  uint32_t above;
-  const uint32_t tk = kth_key(S, (uint32_t)k, cand, true, 0u, &above);
-  const uint32_t need = (uint32_t)k - above;  // keys equal to tk to take, lowest positions first
+  const Kth tk = kth_key(SmemKeys{(int)m, C == 1}, (uint32_t)k, true, 0u);
+  const uint32_t need = (uint32_t)k - tk.above;  // keys equal to Tk to take, lowest positions first
 
-  // 4. this CTA's keys above tk go to the bitmap; its ties are listed
+  // 4. this CTA's keys above Tk go to the bitmap; its ties are listed
   const uint32_t mine = S.cnt_all[r];
   for (uint32_t c0 = 0; c0 < mine; c0 += kThreads) {
     const uint32_t c = c0 + tid;
@@ -526,9 +537,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       key = S.cand_key[c];
       pos = S.cand_pos[c];
     }
-    const bool gt = c < mine && key > tk;
+    const bool gt = c < mine && key > tk.key;
     if (gt) atomicOr(&S.bitmap[(pos - lo) >> 5], 1u << ((pos - lo) & 31));
-    if (c < mine && key == tk) {
+    if (c < mine && key == tk.key) {
       const uint32_t e = atomicAdd(&S.scal[6], 1u);
       S.pool[e] = pos;
     }
@@ -541,30 +552,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     st_cluster_u32(&S.ties_all[r], (uint32_t)tid, S.scal[6]);
   }
   cluster_sync();  // B: every CTA's counts are visible
-  cluster_arrive();  // this CTA reads no other CTA's shared memory from here on
+  cluster_arrive_relaxed();  // this CTA reads no other CTA's shared memory from here on
 
   // output offset of this CTA, and the ties it takes (the lowest positions of the row win)
   uint32_t offset = 0u, ties_before = 0u;
-#pragma unroll
-  for (int q = 0; q < kMaxCluster; ++q) {
-    if (q < (int)r) {
-      const uint32_t ti = S.ties_all[q];
-      const uint32_t qq = need > ties_before ? min(ti, need - ties_before) : 0u;
-      offset += S.above_all[q] + qq;
-      ties_before += ti;
-    }
+  for (int q = 0; q < (int)r; ++q) {
+    const uint32_t ti = S.ties_all[q];
+    const uint32_t qq = need > ties_before ? min(ti, need - ties_before) : 0u;
+    offset += S.above_all[q] + qq;
+    ties_before += ti;
   }
   const uint32_t nties = S.ties_all[r];
   const uint32_t quota = need > ties_before ? min(nties, need - ties_before) : 0u;
   if (quota > 0u) {
+    // take the `quota` lowest tied positions: when not all, select on the complemented position
+    const bool some = quota < nties;
     uint32_t pos_cut = 0xFFFFFFFFu;  // take tied positions <= pos_cut
-    if (quota < nties) {
-      // the `quota` lowest positions among the ties: select on the complemented position
-      const RegKeys<kKPT> tp = load_keys<kKPT>(S.pool, (int)nties, true);
-      pos_cut = ~kth_key(S, quota, tp, true, 0u, nullptr);
+    if (some) {
+      for (uint32_t e = tid; e < nties; e += kThreads) S.pool[e] = ~S.pool[e];
+      __syncthreads();
+      pos_cut = ~kth_key(SmemKeys{(int)nties, false}, quota, true, 0u).key;
     }
     for (uint32_t e = tid; e < nties; e += kThreads) {
-      const uint32_t pos = S.pool[e];
+      const uint32_t pos = some ? ~S.pool[e] : S.pool[e];
       if (pos <= pos_cut) atomicOr(&S.bitmap[(pos - lo) >> 5], 1u << ((pos - lo) & 31));
     }
     __syncthreads();
@@ -576,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t cnt = 0u;
   for (int w = w0; w < w1; ++w) cnt += (uint32_t)__popc(S.bitmap[w]);
   uint32_t total;
-  uint32_t at = offset + block_exclusive_scan(cnt, S.warp_tot, total);
+  uint32_t at = offset + block_exclusive_scan(cnt, total);
   for (int w = w0; w < w1; ++w) {
     uint32_t bits = S.bitmap[w];
     while (bits) {
@@ -586,9 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++at;
     }
   }
-  if (saw_nan) S.scal[4] = 1u;  // benign race: every writer stores 1
-  __syncthreads();
-  if (tid == 0 && S.scal[4]) raise_error(err, DSA_DEVERR_NAN_SCORE);
+  if (tid == 0 && S.scal[4]) raise_error(err, DSA_DEVERR_NAN_SCORE);  // set before the filter's barrier
   cluster_wait();  // no CTA exits while another may still read its shared memory
 }
 

@@ -156,6 +156,19 @@ def test_topk_skewed_and_equal_long_rows():
     assert idx[2].tolist() == list(range(2048))
 
 
+def test_topk_small_tie_groups_in_last_bin():
+    # scores on a coarse grid: the last radix bin of the K-th key holds a few keys, some equal,
+    # and the K-th key may fall anywhere in such a group
+    g = torch.Generator().manual_seed(12)
+    for T, ld, grid in ((1, 32768, 2048.0), (1, 32768, 512.0), (4, 100000, 4096.0), (3, 9000, 256.0)):
+        s = torch.round(torch.randn(T, ld, generator=g) * grid) / grid
+        qpos = [ld - 1 - 13 * t for t in range(T)]
+        for k in (2048, 1999):
+            idx, err = _topk_gpu(s, qpos, k)
+            assert err == 0
+            check_topk(idx, s, qpos, k)
+
+
 def test_topk_nan_in_long_row():
     s = torch.randn(2, 100000)
     s[1, 77777] = float("nan")
