@@ -20,14 +20,20 @@
 // With several key splits per query each unit writes (O / l, LSE) partials that a small combine
 // kernel merges: O = sum_sp exp(LSE_sp - LSE) O_sp, LSE = log sum_sp exp(LSE_sp).
 //
-// Roles (288 threads): warps 0-3 look up the rows of their 16 keys per tile and gather them with
+// Roles (320 threads): warps 0-3 look up the rows of their 16 keys per tile and gather them with
 // TMA (tile::gather4: four rows x 128 bytes per instruction, 128B-swizzled by the copy itself;
 // unused slots point past the pool and read as zeros), and write Q into tensor memory (warp 0
-// lane 0 also loads Q's shared-memory part by TMA); warp 4 owns tensor memory and issues the
-// Q K^T products; warps 5-8 run the softmax and the epilogue (one head row per thread); warp 9
-// issues the P V products.  One thread issues a tensor-core instruction about every 60 cycles,
-// so the two product chains get separate issuing threads: the Q K^T chain of the next tile does
-// not hold back P V, which frees the row-ring stage for the next gather.
+// lane 0 also loads Q's shared-memory part by TMA) after issuing the unit's first gathers, so
+// that both loads are in flight together; warp 4 owns tensor memory and issues the Q K^T
+// products; warps 5-8 run the softmax and the epilogue (one head row per thread); warp 9 issues
+// the P V products.  One thread issues a tensor-core instruction about every 60 cycles, so the two
+// product chains get separate issuing threads: the Q K^T chain of the next tile does not hold
+// back P V, which frees the row-ring stage for the next gather.
+// When every CTA runs a single unit (few queries, latency-bound), Q instead arrives by TMA: the
+// P V thread loads it at the start, dims [0, 320) into the then idle ring stage 1 and P buffer,
+// and the softmax warps, idle until the first S, move each head row from there to tensor memory
+// (per-lane loads of 16-byte pieces of 128 rows would keep L1 busy for microseconds); and the
+// gather warps, idle by the epilogue, store half of O.
 // All waits are bounded; bad indices / block ids set the device error word and are skipped.
 #include <cuda.h>
 #include <math.h>
@@ -62,12 +68,17 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + QS_BYTES;
 constexpr int OFF_P = OFF_K + kStages * K_BYTES;
 constexpr int OFF_BAR = OFF_P + P_BYTES;
-constexpr int NBAR = 2 + 3 * kStages + 5;
+constexpr int NBAR = 2 + 3 * kStages + 8;
 constexpr int OFF_MASK = OFF_BAR + NBAR * 8;                 // valid-row masks [stage][gather warp]
 constexpr int OFF_MISC = OFF_MASK + kStages * kGatherWarps * 4;
-constexpr int BYTES = OFF_MISC + 32;
+constexpr int OFF_STATS = OFF_MISC + 32;                    // 1 / l of each head row (last unit)
+constexpr int BYTES = OFF_STATS + kH * 4;
 constexpr int SMEM = BYTES + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
+
+constexpr int kQStaged = 5;                                  // staged Q: 64-dim boxes through shared memory
+static_assert(kQStaged == 4 + 1 && 4 * Q_CHUNK <= K_BYTES && Q_CHUNK == P_BYTES, "staging: 4 boxes in ring stage 1, 1 in P");
+static_assert(kQStaged + 1 == kTmemQChunks, "the last tensor-memory Q box is loaded directly");
 
 constexpr uint32_t TM_O = 0;       // O half: columns [0, 256)
 constexpr uint32_t TM_S = 256;     // S: [256, 320)
@@ -113,13 +124,15 @@ __device__ __forceinline__ void unit_coords(const Params& p, int u, int& t, int&
 // can be issued a tile apart: the selected position of a slot (kNoSlot when the slot is outside
 // the split or the selection) ...
 constexpr int kNoSlot = -2;
-__device__ __forceinline__ int slot_pos(const Params& p, int t, bool qok, int sp, int slot) {
-  if (!qok || slot >= min(p.k, (sp + 1) * p.ks)) return kNoSlot;
+// (Not gated by the query's validity, so that the load does not wait for the loads behind it:
+// pos_block applies that gate where the position is used, a tile later.)
+__device__ __forceinline__ int slot_pos(const Params& p, int t, int sp, int slot) {
+  if (slot >= min(p.k, (sp + 1) * p.ks)) return kNoSlot;
   return p.idx[(int64_t)t * p.k + slot];
 }
 // ... and the physical block holding it (-1 when unused or out of range; flagged when `report`).
-__device__ __forceinline__ int pos_block(const Params& p, int req, int pos, int ps, bool report) {
-  if (ps == kNoSlot || ps == -1) return -1;
+__device__ __forceinline__ int pos_block(const Params& p, bool qok, int req, int pos, int ps, bool report) {
+  if (!qok || ps == kNoSlot || ps == -1) return -1;
   if (ps < 0 || ps > pos) {
     if (report) raise_error(p.err, DSA_DEVERR_INDEX);
     return -1;
@@ -140,12 +153,89 @@ __device__ __forceinline__ void prefetch_q(const Params& p, int t) {
   for (int off = 0; off < kH * kDqk * 2; off += 16384) prefetch_l2_bulk(src + off, 16384u);
 }
 
+// Staging place of the staged Q's box c (dims [64 c, 64 c + 64), 128 rows, 128B-swizzled,
+// 1024-byte aligned): boxes 0..3 in ring stage 1, box 4 in the P buffer.
+__device__ __forceinline__ uint8_t* q_stage_box(uint8_t* smem, int c) {
+  return c < 4 ? smem + OFF_K + K_BYTES + c * Q_CHUNK : smem + OFF_P;
+}
+
 __device__ __forceinline__ int unit_tiles(const Params& p, int sp) {
   const int first = sp * p.ks;
   const int n = min(p.ks, p.k - first);
   return n > 0 ? (n + kTile - 1) / kTile : 0;
 }
 
+// Rows [32 q, 32 q + 32) of O_v / l (q = this warp's tensor-memory lane quarter), columns
+// [c_lo, c_hi) of the value half (multiples of 64), from tensor memory to the partials (f32, with
+// key splits) or the output (bf16), through a 4 KB staging area: lane i stages its row i (128
+// bytes per block, 16-byte pieces XOR-permuted by i mod 8), then the warp writes rows 4k + lane/8,
+// piece lane mod 8, so that each global store instruction writes four whole 128-byte row pieces.
+// prow / orow: this lane's partial / output row.  have_o false (a unit without rows) stores zeros.
+__device__ __forceinline__ void store_o(const Params& p, uint32_t lane_base, int c_lo, int c_hi, uint8_t* stage,
+                                        float inv, bool have_o, int64_t prow, int64_t orow, int v) {
+  const int lane = threadIdx.x & 31;
+  const int srow = lane >> 3, spiece = lane & 7;
+  const bool f32out = p.nsplit > 1;
+  // write the staged 128-byte block of each of this warp's rows to columns [col, col + 128 B)
+  auto flush = [&](int col) {
+    __syncwarp();
+#pragma unroll
+    for (int k4 = 0; k4 < 8; ++k4) {
+      const int rr = k4 * 4 + srow;  // row within this warp's 32
+      const uint4 x = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((spiece ^ (rr & 7)) << 4));
+      if (f32out)
+        *reinterpret_cast<uint4*>(p.part_o + (prow - lane + rr) * kDv + v * kHalf + col + spiece * 4) = x;
+      else
+        *reinterpret_cast<uint4*>(p.out + (orow - lane + rr) * kDv + v * kHalf + col + spiece * 8) = x;
+    }
+    __syncwarp();
+  };
+#pragma unroll 1
+  for (int c0 = c_lo; c0 < c_hi; c0 += 64) {
+    uint32_t o[64];
+    if (have_o) {
+      tmem_ld16(lane_base + TM_O + c0, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+      tmem_ld16(lane_base + TM_O + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
+      tmem_ld16(lane_base + TM_O + c0 + 32, *reinterpret_cast<uint32_t(*)[16]>(&o[32]));
+      tmem_ld16(lane_base + TM_O + c0 + 48, *reinterpret_cast<uint32_t(*)[16]>(&o[48]));
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int c = 0; c < 64; ++c) o[c] = 0u;
+    }
+    uint8_t* srow_ptr = stage + lane * 128;
+    if (f32out) {
+      // two blocks of 32 f32 columns
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int c = 32 * b + 4 * j;
+          *reinterpret_cast<float4*>(srow_ptr + ((j ^ (lane & 7)) << 4)) =
+              make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
+                          __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
+        }
+        flush(c0 + 32 * b);
+      }
+    } else {
+      // one block of 64 bf16 columns
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 hv = __floats2bfloat162_rn(__uint_as_float(o[8 * j + 2 * e]) * inv,
+                                                          __uint_as_float(o[8 * j + 2 * e + 1]) * inv);
+          pk[e] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        *reinterpret_cast<uint4*>(srow_ptr + ((j ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      flush(c0);
+    }
+  }
+}
+
+template <bool kStagedQ>
 __global__ void __launch_bounds__(kThreads, 1)
     mla_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap lmap,
                   const Params p) {
@@ -165,12 +255,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_empty + 1;              // P written
   uint64_t* pv_done = p_full + 1;              // P V completed
   uint64_t* mma_fin = pv_done + 1;
+  uint64_t* q_first = mma_fin + 1;             // staged Q: all of it in place
+  uint64_t* q_stage = q_first + 1;             // staged Q: dims [0, 320) in shared memory
+  uint64_t* ep_half = q_stage + 1;             // last unit: row statistics published after its last P V
+  float* stats = reinterpret_cast<float*>(smem + OFF_STATS);
   uint32_t* masks = reinterpret_cast<uint32_t*>(smem + OFF_MASK);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int units = p.T * p.nsplit * 2;
+  // kStagedQ (every CTA runs one unit: few queries): Q is staged by TMA in the then idle ring
+  // stage 1 and P buffer and moved to tensor memory by the softmax warps; otherwise the gather
+  // warps copy each unit's Q.  Two instantiations, so that neither carries the other's code.
+  constexpr bool staged_q = kStagedQ;
   griddep_launch_dependents();
 
   if (tid == 0) {
@@ -191,6 +289,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
     mbar_init(mma_fin, 2);  // both issuing threads
+    mbar_init(q_first, 128 + 1);  // softmax threads + the TMA issue
+    mbar_init(q_stage, 1);
+    mbar_init(ep_half, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -229,20 +330,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ntiles = unit_tiles(p, sp);
       const bool mine = lane < kKeysPerWarp;
       const int kslot = sp * p.ks + gw * kKeysPerWarp + lane;
-      int ps_j = mine && ntiles > 0 ? slot_pos(p, t, qok, sp, kslot) : kNoSlot;
-      int ps_j1 = mine && ntiles > 1 ? slot_pos(p, t, qok, sp, kslot + kTile) : kNoSlot;
-      // Q: the previous unit's Q K^T products must be done with it
-      if (ui >= 1 && !(ok = warp_wait(q_empty, (ui - 1) & 1, p.err, abort_flag))) break;
-      tc_fence_after();
-      if (gw == 0 && lane == 0) {
-        mbar_arrive_expect_tx(q_full, QS_BYTES);
-        for (int c = kTmemQChunks; c < kChunks; ++c)
-          tma_load_2d(q_s + (c - kTmemQChunks) * Q_CHUNK, &qmap, q_full, c * 64, t * kH);
-      }
-      {
-        // this thread's head row, dims 0..383, into tensor-memory columns [320, 512)
+      int ps_j = mine && ntiles > 0 ? slot_pos(p, t, sp, kslot) : kNoSlot;
+      int ps_j1 = mine && ntiles > 1 ? slot_pos(p, t, sp, kslot + kTile) : kNoSlot;
+      // Q of the unit (unless staged), once the previous unit's Q K^T products are done with it,
+      // after the unit's first row gathers are issued: the shared-memory part by TMA, and this
+      // thread's head row, dims [0, 384), into tensor-memory columns [320, 512)
+      auto copy_q = [&]() -> bool {
+        if (ui >= 1 && !warp_wait(q_empty, (ui - 1) & 1, p.err, abort_flag)) return false;
+        tc_fence_after();
+        if (gw == 0 && lane == 0) {
+          mbar_arrive_expect_tx(q_full, QS_BYTES);
+          for (int c = kTmemQChunks; c < kChunks; ++c)
+            tma_load_2d(q_s + (c - kTmemQChunks) * Q_CHUNK, &qmap, q_full, c * 64, t * kH);
+        }
         const uint4* src = reinterpret_cast<const uint4*>(p.q + ((int64_t)t * kH + h) * kDqk);
-#pragma unroll
+#pragma unroll 1
         for (int b = 0; b < 2; ++b) {  // 192 dims = 96 columns per batch, all loads in flight
           uint32_t w[96];
 #pragma unroll
@@ -257,15 +359,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(q_full);
-      }
+        return true;
+      };
       if (!qok && tid == 0 && v == 0 && sp == 0) raise_error(p.err, DSA_DEVERR_REQUEST);
-      int blk_j = mine ? pos_block(p, req, pos, ps_j, v == 0) : -1;
+      int blk_j = mine ? pos_block(p, qok, req, pos, ps_j, v == 0) : -1;
       for (int j = 0; j < ntiles; ++j, ++gi) {
         const int s = gi % kStages;
         const int64_t row = blk_j >= 0 ? (int64_t)blk_j * kPage + (ps_j % kPage) : -1;
-        const int blk_j1 = mine && j + 1 < ntiles ? pos_block(p, req, pos, ps_j1, v == 0) : -1;
-        const int ps_j2 = mine && j + 2 < ntiles ? slot_pos(p, t, qok, sp, kslot + (j + 2) * kTile) : kNoSlot;
+        const int blk_j1 = mine && j + 1 < ntiles ? pos_block(p, qok, req, pos, ps_j1, v == 0) : -1;
+        const int ps_j2 = mine && j + 2 < ntiles ? slot_pos(p, t, sp, kslot + (j + 2) * kTile) : kNoSlot;
         if (gi >= kStages && !(ok = warp_wait(&k_empty[s], ((gi / kStages) - 1) & 1, p.err, abort_flag))) break;
+        // a staged Q sits in ring stage 1 until the softmax warps have moved it
+        if constexpr (staged_q)
+          if (gi == 1 && !(ok = warp_wait(q_first, 0, p.err, abort_flag))) break;
         // publish which of this warp's rows are real to the softmax warps
         const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, row >= 0) & ((1u << kKeysPerWarp) - 1u);
         if (lane == 0) {
@@ -291,6 +397,20 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_gather4(stage + c * K_CHUNK + g4 * 512, &lmap, &k_full[s], c * 64, r0, r1, r2, r3);
           }
         }
+        if constexpr (!staged_q)
+          if (j == 0 && !(ok = copy_q())) break;
+      }
+      if constexpr (!staged_q)
+        if (ok && ntiles == 0) ok = copy_q();
+      if (ok && u + (int)gridDim.x >= units) {
+        // the CTA's last unit: columns [128, 256) of O_v / l, once the softmax warps have published
+        // 1 / l (after the unit's last P V, which also frees the row ring for the staging)
+        if (!(ok = warp_wait(ep_half, 0, p.err, abort_flag))) break;
+        tc_fence_after();
+        const int64_t orow = (int64_t)t * kH + h;
+        const int64_t prow = ((int64_t)t * p.nsplit + sp) * kH + h;
+        store_o(p, my_lanes, kHalf / 2, kHalf, k_ring + gw * 4096, stats[h], ntiles > 0, prow, orow, v);
+        tc_fence_before();
       }
     }
     if (!ok && lane == 0) {
@@ -310,7 +430,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         int t, sp, v;
         unit_coords(p, u, t, sp, v);
         const int ntiles = unit_tiles(p, sp);
-        if (!(ok = mbar_wait(q_full, ui & 1, p.err, abort_flag))) break;
+        if constexpr (staged_q) {
+          if (!(ok = mbar_wait(q_first, 0, p.err, abort_flag))) break;
+        } else {
+          if (!(ok = mbar_wait(q_full, ui & 1, p.err, abort_flag))) break;
+        }
         if (ntiles == 0) mma_commit(q_empty);
         for (int j = 0; j < ntiles; ++j) {
           const int g = gi + j, s = g % kStages;
@@ -341,6 +465,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kPvWarp) {
     // ------------------------------------------------------------------ P V issuer
     if (lane == 0) {
+      if constexpr (staged_q) {
+        // the unit's Q by TMA: dims [384, 576) to their place, dims [0, 320) staged in ring stage 1
+        // (64-dim boxes 0..3) and the P buffer (box 4) for the softmax warps
+        int t0, sp0, v0;
+        unit_coords(p, blockIdx.x, t0, sp0, v0);
+        mbar_arrive_expect_tx(q_first, QS_BYTES);
+        for (int c = kTmemQChunks; c < kChunks; ++c)
+          tma_load_2d(q_s + (c - kTmemQChunks) * Q_CHUNK, &qmap, q_first, c * 64, t0 * kH);
+        mbar_arrive_expect_tx(q_stage, kQStaged * Q_CHUNK);
+        for (int c = 0; c < kQStaged; ++c)
+          tma_load_2d(q_stage_box(smem, c), &qmap, q_stage, c * 64, t0 * kH);
+      }
       const uint32_t idesc_o = idesc_f16(1u, 1u, 128u, (uint32_t)kHalf);  // O: B (V) MN-major
       // P [128 x 64] K-major, no swizzle: 8x16-byte core matrices 128 B apart along K and 1024 B
       // apart along M; one K step (16 keys) is two core matrices = 256 bytes
@@ -379,6 +515,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // head row
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    if constexpr (staged_q) {
+      // the staged Q, head row r, dims [0, 384) into tensor-memory columns [320, 512): dims
+      // [0, 320) from the staged 128B-swizzled boxes (16-byte piece j of row r sits at piece
+      // j ^ (r mod 8)), dims [320, 384) straight from global memory
+      int t0, sp0, v0;
+      unit_coords(p, blockIdx.x, t0, sp0, v0);
+      const uint4* src = reinterpret_cast<const uint4*>(p.q + ((int64_t)t0 * kH + r) * kDqk) + 5 * 8;
+      uint32_t w[32];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint4 x = __ldg(src + e);
+        w[4 * e] = x.x; w[4 * e + 1] = x.y; w[4 * e + 2] = x.z; w[4 * e + 3] = x.w;
+      }
+      const bool qs_ok = mbar_wait(q_stage, 0, p.err, abort_flag);
+#pragma unroll 1
+      for (int c = 0; c < kQStaged && qs_ok; ++c) {
+        const uint8_t* row = q_stage_box(smem, c) + r * 128;
+        uint32_t x[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 y = *reinterpret_cast<const uint4*>(row + ((j ^ (r & 7)) << 4));
+          x[4 * j] = y.x; x[4 * j + 1] = y.y; x[4 * j + 2] = y.z; x[4 * j + 3] = y.w;
+        }
+        tmem_st16(lane_base + TM_Q + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&x[0]));
+        tmem_st16(lane_base + TM_Q + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&x[16]));
+      }
+      tmem_st16(lane_base + TM_Q + kQStaged * 32, *reinterpret_cast<uint32_t(*)[16]>(&w[0]));
+      tmem_st16(lane_base + TM_Q + kQStaged * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&w[16]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(q_first);
+    }
     int gi = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
@@ -473,69 +641,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t orow = (int64_t)t * kH + r;
       const int64_t prow = ((int64_t)t * p.nsplit + sp) * kH + r;
       // O / l leaves through this warp's 4 KB quarter of the P buffer (free: the last P V has
-      // completed), so that each global store instruction writes four whole 128-byte row pieces:
-      // lane i stages its row i (128 bytes per block, 16-byte pieces XOR-permuted by i mod 8),
-      // then the warp writes rows 4k + lane/8, piece lane mod 8.
-      uint8_t* stage = p_s + quarter * 4096;
-      const int srow = lane >> 3, spiece = lane & 7;
-      const bool f32out = p.nsplit > 1;
-      // write the staged 128-byte block of each of this warp's rows to columns [col, col + 128 B)
-      auto flush = [&](int col) {
-        __syncwarp();
-#pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-          const int rr = k4 * 4 + srow;  // row within this warp's 32
-          const uint4 x = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((spiece ^ (rr & 7)) << 4));
-          if (f32out)
-            *reinterpret_cast<uint4*>(p.part_o + (prow - lane + rr) * kDv + v * kHalf + col + spiece * 4) = x;
-          else
-            *reinterpret_cast<uint4*>(p.out + (orow - lane + rr) * kDv + v * kHalf + col + spiece * 8) = x;
-        }
-        __syncwarp();
-      };
-#pragma unroll 1
-      for (int c0 = 0; c0 < kHalf; c0 += 64) {
-        uint32_t o[64];
-        if (ntiles > 0) {
-          tmem_ld16(lane_base + TM_O + c0, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
-          tmem_ld16(lane_base + TM_O + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
-          tmem_ld16(lane_base + TM_O + c0 + 32, *reinterpret_cast<uint32_t(*)[16]>(&o[32]));
-          tmem_ld16(lane_base + TM_O + c0 + 48, *reinterpret_cast<uint32_t(*)[16]>(&o[48]));
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) o[c] = 0u;
-        }
-        uint8_t* srow_ptr = stage + lane * 128;
-        if (f32out) {
-          // two blocks of 32 f32 columns
-#pragma unroll
-          for (int b = 0; b < 2; ++b) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int c = 32 * b + 4 * j;
-              *reinterpret_cast<float4*>(srow_ptr + ((j ^ (lane & 7)) << 4)) =
-                  make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
-                              __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
-            }
-            flush(c0 + 32 * b);
-          }
-        } else {
-          // one block of 64 bf16 columns
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const __nv_bfloat162 hv = __floats2bfloat162_rn(__uint_as_float(o[8 * j + 2 * e]) * inv,
-                                                              __uint_as_float(o[8 * j + 2 * e + 1]) * inv);
-              pk[e] = *reinterpret_cast<const uint32_t*>(&hv);
-            }
-            *reinterpret_cast<uint4*>(srow_ptr + ((j ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          }
-          flush(c0);
-        }
+      // completed).  In the CTA's last unit the gather warps, idle by then, store the columns
+      // [128, 256) of the half: they get 1 / l through shared memory once the last P V is done.
+      const bool last = u + (int)gridDim.x >= units;
+      if (last) {
+        stats[r] = inv;
+        mbar_arrive(ep_half);
       }
+      store_o(p, lane_base, 0, last ? kHalf / 2 : kHalf, p_s + quarter * 4096, inv, ntiles > 0, prow, orow, v);
       if (v == 0) {
         if (p.nsplit == 1) {
           if (p.lse) p.lse[orow] = lse;
@@ -697,13 +810,14 @@ cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_
     p.part_o = static_cast<float*>(a.workspace);
     p.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) + ((o + 255) / 256) * 256);
   }
-  cudaError_t e = cudaFuncSetAttribute(mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-  if (e != cudaSuccess) return e;
   const int units = T * nsplit * 2;
   const int grid = units < num_sms ? units : num_sms;
+  auto kernel = units <= grid ? mla_tc_kernel<true> : mla_tc_kernel<false>;  // one unit per CTA: staged Q
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (e != cudaSuccess) return e;
   cudaLaunchAttribute attrs[2];
   const cudaLaunchConfig_t cfg = launch_config(dim3(grid), dim3(kThreads), SMEM, s, attrs);
-  e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, qmap, lmap, p);
+  e = cudaLaunchKernelEx(&cfg, kernel, qmap, lmap, p);
   if (e != cudaSuccess || nsplit == 1) return e;
   cudaLaunchAttribute cattrs[2];
   const cudaLaunchConfig_t ccfg = launch_config(dim3(T, kH), dim3(kCombThreads), 0, s, cattrs);
