@@ -34,6 +34,25 @@ def test_decode_ragged_batch(key_dtype):
     parity_case(x, kind=key_dtype)
 
 
+@pytest.mark.parametrize("lens", [[6000], [3000, 2500, 7000]])
+def test_decode_few_queries_many_splits(lens):
+    # one or three queries at K = 2048: the rows of each query split across many CTAs (one 64-row
+    # tile each), one unit per CTA with Q staged through shared memory, partials merged by the combine
+    spec = _spec(lens, seed=15)
+    x = to_dev(di.generate(spec, "cpu"))
+    parity_case(x, kind="bf16")
+
+
+def test_decode_split_partials_and_combine():
+    # 75 decode queries of one request: more (query, split) units than SMs, so the splits leave
+    # partials in the workspace and the combine kernel merges them
+    ctx, n = 2200, 75
+    spec = di.Spec("many", lens=[ctx], q_req=[0] * n, q_pos=[ctx - n + i for i in range(n)], seed=16)
+    x = to_dev(di.generate(spec, "cpu"))
+    assert dsa.dsa_mla_workspace_size(spec.T, spec.H, spec.d_v, spec.k) > 0
+    parity_case(x, queries=range(0, n, 7), kind="bf16")  # the oracle on every 7th query
+
+
 def test_decode_small_k_many_tiles():
     spec = _spec([1000, 777], k=100, seed=12)
     x = to_dev(di.generate(spec, "cpu"))
