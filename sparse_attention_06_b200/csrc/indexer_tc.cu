@@ -57,7 +57,12 @@ struct Cfg {
   static constexpr int OPS = TMEM_A ? 4 : FP8 ? 2 : (NQ == 1 ? 5 : 4);  // operand stages
   static constexpr int STS = FP8 ? (NQ == 1 ? 8 : 4) : 0;     // fp8 staging stages
   static constexpr int QS = NQ == 1 ? 2 : 1;                  // query slots
-  static constexpr int TIS = NQ == 1 ? 24 : 16;               // tile-info ring entries
+  static constexpr int TIS = NQ == 1 ? (FP8 ? 48 : 24) : 16;  // tile-info ring entries
+  // Tiles whose info the producer publishes in one lane-parallel pass.  A ring entry is free again
+  // once the epilogue has looked at its previous tile, which it does after finishing the tile LOOK
+  // of its own tiles earlier; so a pass never waits on the epilogue while TIS - PUB - LOOK * tstep
+  // covers the tiles in flight (at most STS + OPS + 2), and it can never wait on tiles of its own.
+  static constexpr int PUB = NQ == 1 && FP8 ? 32 : 8;
   // Tiles (of its own) an epilogue warp reads ahead in the tile-info ring.  The producer runs at
   // most STS + OPS + 2 tiles (e4m3) or OPS + 2 tiles (bf16) ahead of the epilogue's last finished
   // tile, so the distance stays below that; only e4m3 needs it (its scale copies).
@@ -89,6 +94,10 @@ struct Cfg {
   // has seen the stage's previous phase: with two issuers alternating tiles, every stage must
   // belong to one of them (an even number of stages).
   static_assert(MMA_WARPS == 1 || OPS % 2 == 0, "operand stages must not alternate between issuers");
+  // a publication pass waits only on tiles issued before it, and not while the pipeline is full
+  static_assert(TIS + LOOK * (EPI_ALT ? 2 : 1) >= PUB, "tile-info ring too small for a publication pass");
+  static_assert(TIS + LOOK * (EPI_ALT ? 2 : 1) - PUB >= STS + OPS + 2, "a publication pass would wait on the pipeline");
+  static_assert(PUB <= 32, "one lane per tile");
   // shared-memory carve-up (offsets from a 1024-aligned base)
   static constexpr int OFF_OP = 0;
   static constexpr int OFF_ST = OFF_OP + (TMEM_A ? 0 : OPS * OP_BYTES);
@@ -97,7 +106,8 @@ struct Cfg {
   static constexpr int OFF_SC = OFF_W + EPI_WARPS * EPI_NQ * kHeads * 4;  // w, one copy per epilogue warp
   static constexpr int OFF_PR = OFF_SC + (FP8 ? TIS * kTileKeys * 4 : 0);  // key scales of ring tiles
   static constexpr int OFF_TI = OFF_PR + TIS * kTileKeys;                  // row present, per ring tile
-  static constexpr int OFF_BAR = OFF_TI + TIS * 8;                         // block ids of ring tiles
+  static constexpr int OFF_BT = OFF_TI + TIS * 8;                          // block ids of ring tiles
+  static constexpr int OFF_BAR = OFF_BT + 32 * 16;                         // the producer's batch table
   static constexpr int NBAR = 2 * OPS + 2 * STS + 3 * QS + 4 + 1 + 2 * TIS;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 64;
@@ -280,6 +290,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
   float* sc_ring = reinterpret_cast<float*>(smem + C::OFF_SC);  // [TIS][128] (e4m3) key scales
   uint8_t* pr_ring = smem + C::OFF_PR;                           // [TIS][128] row's page present
   int2* ti_ring = reinterpret_cast<int2*>(smem + C::OFF_TI);     // [TIS] block ids of the pages
+  int4* batch_tab = reinterpret_cast<int4*>(smem + C::OFF_BT);   // [32] producer: (block ids, group) per tile
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* op_full = bars;
   uint64_t* op_empty = op_full + C::OPS;
@@ -380,67 +391,81 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
         n_r1 = n_grp >= 0 ? lookup_block(p, mG, mj, 1) : -1;
       };
       fetch();
-      int last = -1, m = -1;
-      int64_t i = 0;
+      int last = -1, m = -1;  // (lane 0) group of the last query tile issued, query tiles issued
+      int64_t i = 0;          // tiles whose copies were issued (the first tile of the batch below)
       bool ok = true;
       while (ok && n_cnt > 0) {
-        const int cnt = n_cnt, my_grp = n_grp, r0 = n_r0, r1 = n_r1;
-        fetch();
-        for (int l = 0; l < cnt; ++l) {
-          const int grp = __shfl_sync(0xFFFFFFFFu, my_grp, l);
-          const int raw0 = __shfl_sync(0xFFFFFFFFu, r0, l);
-          const int raw1 = __shfl_sync(0xFFFFFFFFu, r1, l);
-          if (lane == 0) {
-            const int b0 = check_block(p, raw0);
-            const int b1 = check_block(p, raw1);
-            {
-              // tile info for the epilogue: the block ids of the tile's pages (-1: absent).  It is
-              // published before any wait of this tile below, which depend on the epilogue.
-              const int c = (int)(i % C::TIS), cu = (int)(i / C::TIS);
-              if (cu >= 1 && !(ok = mbar_wait(&ti_empty[c], (cu - 1) & 1, p.err, abort_flag))) goto issued;
-              ti_ring[c] = make_int2(b0, b1);
+        const int cnt = n_cnt;
+        // this lane's tile of the batch (tile i + lane): block ids checked, into the batch table
+        const int b0 = lane < cnt ? check_block(p, n_r0) : -1;
+        const int b1 = lane < cnt ? check_block(p, n_r1) : -1;
+        batch_tab[lane] = make_int4(b0, b1, n_grp, 0);
+        fetch();  // the next batch's lookups, in flight while this one is issued
+        __syncwarp();
+        for (int l0 = 0; l0 < cnt && ok; l0 += C::PUB) {
+          const int n = min(C::PUB, cnt - l0);
+          // tile info of tiles l0 .. l0 + n - 1 of the batch, one lane each: published before any
+          // wait of these tiles below, which depend on the epilogue
+          bool lok = true;
+          if (lane < n) {
+            const int4 e = batch_tab[l0 + lane];
+            const int64_t x = i + l0 + lane;
+            const int c = (int)(x % C::TIS), cu = (int)(x / C::TIS);
+            if (cu >= 1 && !mbar_wait(&ti_empty[c], (cu - 1) & 1, p.err, abort_flag)) {
+              lok = false;
+            } else {
+              ti_ring[c] = make_int2(e.x, e.y);
               mbar_arrive(&ti_full[c]);
             }
-            if (grp != last) {
-              const int mm = m + 1;  // m counts the query tiles issued so far
-              const int slot = mm % C::QS, use = mm / C::QS;
-              if (use >= 1 && !(ok = mbar_wait(&q_empty[slot], (use - 1) & 1, p.err, abort_flag))) goto issued;
-              mbar_arrive_expect_tx(&q_full[slot], C::Q_BYTES);
-              uint8_t* qd = q_slots + slot * C::Q_BYTES;
-              tma_load_2d(qd, &qmap, &q_full[slot], 0, grp * NQ * kHeads);
-              tma_load_2d(qd + C::Q_CHUNK, &qmap, &q_full[slot], 64, grp * NQ * kHeads);
-              m = mm;
-              last = grp;
-            }
-            {
+          }
+          ok = __all_sync(0xFFFFFFFFu, lok);
+          if (!ok) break;
+          // the query tiles and key copies of these tiles, in order, from lane 0
+          int64_t issued = i + l0;
+          if (lane == 0) {
+            for (int l = l0; l < l0 + n; ++l) {
+              const int4 e = batch_tab[l];
+              const int grp = e.z, t0 = e.x, t1 = e.y;
+              if (grp != last) {
+                const int mm = m + 1;  // m counts the query tiles issued so far
+                const int slot = mm % C::QS, use = mm / C::QS;
+                if (use >= 1 && !(ok = mbar_wait(&q_empty[slot], (use - 1) & 1, p.err, abort_flag))) break;
+                mbar_arrive_expect_tx(&q_full[slot], C::Q_BYTES);
+                uint8_t* qd = q_slots + slot * C::Q_BYTES;
+                tma_load_2d(qd, &qmap, &q_full[slot], 0, grp * NQ * kHeads);
+                tma_load_2d(qd + C::Q_CHUNK, &qmap, &q_full[slot], 64, grp * NQ * kHeads);
+                m = mm;
+                last = grp;
+              }
               if constexpr (FP8) {
-                const int s = (int)(i % C::STS), use = (int)(i / C::STS);
-                if (use >= 1 && !(ok = mbar_wait(&st_empty[s], (use - 1) & 1, p.err, abort_flag))) goto issued;
-                mbar_arrive_expect_tx(&st_full[s], (b0 >= 0 ? 8192u : 0u) + (b1 >= 0 ? 8192u : 0u));
-                uint8_t* dst = st_ring + s * C::ST_BYTES;
-                if (b0 >= 0) tma_load_2d(dst, &kmap, &st_full[s], 0, b0 * kPage);
-                if (b1 >= 0) tma_load_2d(dst + 8192, &kmap, &st_full[s], 0, b1 * kPage);
+                const int st = (int)(issued % C::STS), use = (int)(issued / C::STS);
+                if (use >= 1 && !(ok = mbar_wait(&st_empty[st], (use - 1) & 1, p.err, abort_flag))) break;
+                mbar_arrive_expect_tx(&st_full[st], (t0 >= 0 ? 8192u : 0u) + (t1 >= 0 ? 8192u : 0u));
+                uint8_t* dst = st_ring + st * C::ST_BYTES;
+                if (t0 >= 0) tma_load_2d(dst, &kmap, &st_full[st], 0, t0 * kPage);
+                if (t1 >= 0) tma_load_2d(dst + 8192, &kmap, &st_full[st], 0, t1 * kPage);
               } else {
-                const int s = (int)(i % C::OPS), use = (int)(i / C::OPS);
-                if (use >= 1 && !(ok = mbar_wait(&op_empty[s], (use - 1) & 1, p.err, abort_flag))) goto issued;
-                mbar_arrive_expect_tx(&op_full[s], (b0 >= 0 ? 16384u : 0u) + (b1 >= 0 ? 16384u : 0u));
-                uint8_t* dst = op_ring + s * C::OP_BYTES;
-                if (b0 >= 0) {
-                  tma_load_2d(dst, &kmap, &op_full[s], 0, b0 * kPage);
-                  tma_load_2d(dst + C::CHUNK_BYTES, &kmap, &op_full[s], 64, b0 * kPage);
+                const int st = (int)(issued % C::OPS), use = (int)(issued / C::OPS);
+                if (use >= 1 && !(ok = mbar_wait(&op_empty[st], (use - 1) & 1, p.err, abort_flag))) break;
+                mbar_arrive_expect_tx(&op_full[st], (t0 >= 0 ? 16384u : 0u) + (t1 >= 0 ? 16384u : 0u));
+                uint8_t* dst = op_ring + st * C::OP_BYTES;
+                if (t0 >= 0) {
+                  tma_load_2d(dst, &kmap, &op_full[st], 0, t0 * kPage);
+                  tma_load_2d(dst + C::CHUNK_BYTES, &kmap, &op_full[st], 64, t0 * kPage);
                 }
-                if (b1 >= 0) {
-                  tma_load_2d(dst + 8192, &kmap, &op_full[s], 0, b1 * kPage);
-                  tma_load_2d(dst + C::CHUNK_BYTES + 8192, &kmap, &op_full[s], 64, b1 * kPage);
+                if (t1 >= 0) {
+                  tma_load_2d(dst + 8192, &kmap, &op_full[st], 0, t1 * kPage);
+                  tma_load_2d(dst + C::CHUNK_BYTES + 8192, &kmap, &op_full[st], 64, t1 * kPage);
                 }
               }
+              ++issued;
             }
-            ++i;
-          issued:;
           }
           ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-          if (!ok) break;
+          if (!ok) i = __shfl_sync(0xFFFFFFFFu, issued, 0);
         }
+        if (ok) i += cnt;
+        __syncwarp();  // the batch table is rewritten by the next batch
       }
       if (!ok && lane == 0) {
         // give up: let the copies already issued land before the CTA's memory goes away
