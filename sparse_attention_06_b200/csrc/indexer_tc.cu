@@ -687,19 +687,24 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
         tmem_wait_st();
         tc_fence_before();
       } else {
-        // 8 codes -> one 16-byte chunk of the swizzled operand: the 8 threads of a quarter-warp
-        // fill the 8 chunks of one 128-byte row, so the stores hit distinct banks
+        // 16 codes -> two 16-byte chunks (2 c16, 2 c16 + 1) of the swizzled operand; the 8 threads of a
+        // quarter-warp cover one 128-byte row of codes, so the loads are contiguous, and the threads
+        // of the second 64-dim block store their odd chunk first, so that each store instruction
+        // hits eight distinct 16-byte bank groups
         uint8_t* dst = op_ring + so * C::OP_BYTES;
-        constexpr int kSteps = (kTileKeys * kDim / 8) / (32 * (C::CONV_WARPS > 0 ? C::CONV_WARPS : 1));
+        constexpr int kSteps = (kTileKeys * kDim / 16) / (32 * (C::CONV_WARPS > 0 ? C::CONV_WARPS : 1));
 #pragma unroll 4
         for (int k = 0; k < kSteps; ++k) {
-          const int piece = ct + 32 * C::CONV_WARPS * k;  // 8-byte piece: row piece/16, codes 8 (piece%16) ..
-          const int row = piece >> 4, c8 = piece & 15;
-          const uint2 in = *reinterpret_cast<const uint2*>(src + row * 128 + c8 * 8);
-          uint4 o;
-          e4m3x4_to_f16x4(in.x, o.x, o.y);
-          e4m3x4_to_f16x4(in.y, o.z, o.w);
-          *reinterpret_cast<uint4*>(dst + (c8 >> 3) * C::CHUNK_BYTES + sw128_offset(row, c8 & 7)) = o;
+          const int piece = ct + 32 * C::CONV_WARPS * k;  // 16-byte piece: row piece/8, codes 16 (piece%8) ..
+          const int row = piece >> 3, c16 = piece & 7;
+          const uint4 in = *reinterpret_cast<const uint4*>(src + row * 128 + c16 * 16);
+          uint4 o0, o1;
+          e4m3x16_to_f16(in, o0, o1);
+          uint8_t* blk = dst + (c16 >> 2) * C::CHUNK_BYTES;
+          const uint32_t ch = (uint32_t)(2 * c16) & 7u;
+          const bool odd_first = c16 >= 4;
+          *reinterpret_cast<uint4*>(blk + sw128_offset(row, ch + (odd_first ? 1u : 0u))) = odd_first ? o1 : o0;
+          *reinterpret_cast<uint4*>(blk + sw128_offset(row, ch + (odd_first ? 0u : 1u))) = odd_first ? o0 : o1;
         }
         fence_proxy_async_smem();
       }
