@@ -693,7 +693,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
         // hits eight distinct 16-byte bank groups
         uint8_t* dst = op_ring + so * C::OP_BYTES;
         constexpr int kSteps = (kTileKeys * kDim / 16) / (32 * (C::CONV_WARPS > 0 ? C::CONV_WARPS : 1));
-#pragma unroll 4
+#pragma unroll
         for (int k = 0; k < kSteps; ++k) {
           const int piece = ct + 32 * C::CONV_WARPS * k;  // 16-byte piece: row piece/8, codes 16 (piece%8) ..
           const int row = piece >> 3, c16 = piece & 7;
