@@ -72,8 +72,6 @@ struct Cfg {
   static constexpr int ST_BYTES = kTileKeys * kDim;           // 16 KB fp8 key tile
   static constexpr int Q_BYTES = N * kDim * 2;
   static constexpr int Q_CHUNK = N * 128;
-  static constexpr int A_COLS = kDim / 2;                     // TMEM columns of one f16 key tile
-  static constexpr int A_COL0 = 2 * N;                        // first A stage (TMEM_A)
   static constexpr int TMEM_COLS = TMEM_A ? 512 : 2 * N;
   // Epilogue: two sets of four warps (each set covers the 128 TMEM lanes).  With one query per
   // tile the sets take alternate tiles (set s owns accumulator s); with four queries both sets
@@ -203,6 +201,11 @@ struct Walk {
 // visible key, -2 when its logical block is past the table.  Only the load; check_block() judges
 // the value when it is used, so that the load stays in flight until then.  A negative table entry
 // for a page with visible keys is an error like any other id outside the pool (it reads as -3).
+// TMEM_A: tensor-memory column of converted key-tile stage s (after the two accumulators of N
+// columns; one f16 key tile = 128 dims = 64 columns)
+template <int N>
+__device__ __forceinline__ uint32_t a_stage_col(int s) { return (uint32_t)(2 * N + s * (kDim / 2)); }
+
 __device__ __forceinline__ int lookup_block(const Params& p, const Group& G, int j, int pg) {
   const int first = j * kTileKeys + pg * kPage;
   if (G.tiles == 0 || first >= G.nmax) return -1;
@@ -513,7 +516,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
         constexpr uint64_t ac = C::CHUNK_BYTES >> 4, bc = C::Q_CHUNK >> 4;
         if constexpr (C::TMEM_A) {
           // A = the f16 key tile in tensor memory: one K step of 16 dims = 8 columns
-          const uint32_t at = tmem_base + (uint32_t)(C::A_COL0 + s * C::A_COLS);
+          const uint32_t at = tmem_base + a_stage_col<C::N>(s);
           umma_ts<0>(d, at, bd, idesc);
           umma_ts<1>(d, at + 8, bd + 2, idesc);
           umma_ts<1>(d, at + 16, bd + 4, idesc);
@@ -669,7 +672,7 @@ __global__ void __launch_bounds__(Cfg<NQ, FP8>::THREADS, 1)
         tc_fence_after();
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        const uint32_t ta = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(C::A_COL0 + so * C::A_COLS);
+        const uint32_t ta = tmem_base + ((uint32_t)(quarter * 32) << 16) + a_stage_col<C::N>(so);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // dims [64 h, 64 h + 64) -> 32 columns
           uint32_t f[32];
