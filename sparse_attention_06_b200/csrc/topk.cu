@@ -12,8 +12,10 @@
 //
 //   1. Threshold.  Every CTA reads the same strided sample of the row (8-score chunks; the loads
 //      of its own slice are already in flight) and finds, by radix steps of 12-bit digits, a key
-//      tau with at least js sample keys >= tau, where js is the sample rank expected to leave
-//      ~1.15 K + 4 sqrt(K) scores of the row at or above tau.  Rows of at most kCap positions take
+//      tau with at least js sample keys >= tau, js = rk + 4 sqrt(rk) + 8 where rk is the sample
+//      rank of the row's K-th score: the count of sample keys above that score is about binomial
+//      with mean rk, so fewer than K candidates (and the exact path below) needs a deviation of
+//      more than four standard deviations (~1e-6 per row).  Rows of at most kCap positions take
 //      every score (no threshold).
 //   2. Filter.  One coalesced pass over the slice appends every (key, position) with
 //      score >= tau to shared memory (one shared atomic per warp and 256 scores), and the CTA
@@ -451,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int e = 0; e < kSPT; ++e) S.pool[tid + e * kThreads] = order_key(sv[e], saw_nan);
     __syncthreads();  // sample keys and cleared histograms visible
     const float rk = (float)k * (float)kSample / (float)n;  // sample rank of the row's K-th score
-    int js = (int)ceilf(1.15f * rk + 4.f * sqrtf(rk) + 8.f);
+    int js = (int)ceilf(rk + 4.f * sqrtf(rk) + 8.f);
     js = min(js, kSample);
     tau_f = key_to_float(kth_key(SmemKeys{kSample, false}, (uint32_t)js, false, (uint32_t)(js / 8 + 2)).key);
   } else {
