@@ -188,6 +188,20 @@ def test_topk_small_tie_groups_in_last_bin():
             check_topk(idx, s, qpos, k)
 
 
+def test_topk_threshold_from_a_misleading_sample():
+    # the strided sample (8-score chunks at multiples of n / 512) sees only large scores, so its
+    # threshold leaves fewer than K candidates and the selection falls back to its exact path
+    g = torch.Generator().manual_seed(13)
+    n = 32768
+    s = torch.randn(1, n, generator=g)
+    pos = torch.arange(512).repeat_interleave(8) * (n // 512) + torch.arange(8).repeat(512)
+    s[0, pos] = 10.0 + torch.rand(pos.numel(), generator=g)
+    for k in (2048, 1000):
+        idx, err = _topk_gpu(s, [n - 1], k)
+        assert err == 0
+        check_topk(idx, s, [n - 1], k)
+
+
 def test_topk_nan_in_long_row():
     s = torch.randn(2, 100000)
     s[1, 77777] = float("nan")
