@@ -124,6 +124,15 @@ __device__ __forceinline__ uint32_t ld_cluster_u32(const uint32_t* local, uint32
   return v;
 }
 
+// Four consecutive 32-bit words (16-byte aligned) from the shared memory of CTA `rank`.
+__device__ __forceinline__ uint4 ld_cluster_u32x4(const uint32_t* local, uint32_t rank) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(cluster_addr(local, rank)));
+  return v;
+}
+
 // 32-bit store into the shared memory of CTA `rank`; made visible by the next cluster barrier.
 __device__ __forceinline__ void st_cluster_u32(uint32_t* local, uint32_t rank, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr(local, rank)), "r"(v) : "memory");
@@ -510,19 +519,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // 3. exact K-th key among the row's candidates (gathered from every CTA of the cluster into the
-  //    pool, CTA by CTA; the first 512 of each CTA's keys are loaded at once)
+  //    pool, CTA by CTA, four keys per remote load; the first 2048 of each CTA's keys at once)
   if (C > 1) {
-    uint32_t val[kMaxCluster];
+    constexpr uint32_t kSpan = 4 * kThreads;
+    const uint32_t i0 = 4u * (uint32_t)tid;
+    uint4 val[kMaxCluster];
 #pragma unroll
     for (int q = 0; q < kMaxCluster; ++q) {
       const uint32_t cq = q < (int)C ? S.cnt_all[q] : 0u;
-      val[q] = (uint32_t)tid < cq ? ld_cluster_u32(&S.cand_key[tid], (uint32_t)q) : 0u;
+      val[q] = i0 < cq ? ld_cluster_u32x4(&S.cand_key[i0], (uint32_t)q) : make_uint4(0u, 0u, 0u, 0u);
     }
     uint32_t pre = 0u;
-    for (int q = 0; q < (int)C; ++q) {
-      const uint32_t cq = S.cnt_all[q];
-      if ((uint32_t)tid < cq) S.pool[pre + tid] = val[q];
-      for (uint32_t i = tid + kThreads; i < cq; i += kThreads) S.pool[pre + i] = ld_cluster_u32(&S.cand_key[i], (uint32_t)q);
+#pragma unroll
+    for (int q = 0; q < kMaxCluster; ++q) {
+      const uint32_t cq = q < (int)C ? S.cnt_all[q] : 0u;
+      for (uint32_t i = i0; i < cq; i += kSpan) {
+        const uint4 x = i == i0 ? val[q] : ld_cluster_u32x4(&S.cand_key[i], (uint32_t)q);
+        S.pool[pre + i] = x.x;  // entries at or past cq are stale: not copied
+        if (i + 1 < cq) S.pool[pre + i + 1] = x.y;
+        if (i + 2 < cq) S.pool[pre + i + 2] = x.z;
+        if (i + 3 < cq) S.pool[pre + i + 3] = x.w;
+      }
       pre += cq;
     }
     __syncthreads();
