@@ -19,9 +19,9 @@
 //
 // One persistent CTA per SM walks a contiguous range of the (query group, key tile) list.  Roles:
 //   warp 0      producer: looks up the block ids of the next 32 tiles at once (one lane per tile,
-//               the following batch already in flight), then issues the TMA copies of key pages
-//               and query tiles into 128B-swizzled shared memory and records each tile's block
-//               ids in a tile-info ring
+//               the following batch already in flight), checks them and publishes 8-32 tiles'
+//               block ids in a tile-info ring in one lane-parallel pass, then (lane 0) issues the
+//               TMA copies of key pages and query tiles into 128B-swizzled shared memory
 //   warp 1      TMEM allocation and the thread that issues tcgen05.mma / tcgen05.commit (for e4m3
 //               keys with one query per tile, of the even tiles; the last warp issues the odd ones)
 //   epilogue    8 warps in two sets (alternate tiles with one query per tile, else half of the
