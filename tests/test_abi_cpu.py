@@ -84,3 +84,21 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(dsa, "_lib", None)
     with pytest.raises(dsa.DsaLibraryMissing):
         dsa.load_library()
+
+
+def test_mla_split_plan_and_workspace(lib):
+    # The decode plan of the tensor-core MLA: key splits per query chosen by the library's cost
+    # model for a 148-SM B200 (the SM count the library assumes when no device answers), and the
+    # workspace of their f32 partials: T * nsplit * 128 * (512 + 1) floats in two 256-byte aligned
+    # parts.  A query alone spreads its 32 row tiles over 32 CTA pairs; a batch that already fills
+    # the SMs takes no split (and needs no workspace).
+    def ws(T, nsplit):
+        o = T * nsplit * 128 * 512 * 4
+        l = T * nsplit * 128 * 4
+        return ((o + 255) // 256) * 256 + ((l + 255) // 256) * 256
+    for T, nsplit in ((1, 32), (3, 16), (8, 8), (16, 4), (75, 2), (100, 2)):
+        assert lib.dsa_mla_workspace_size(T, 128, 512, 2048) == ws(T, nsplit), T
+    assert lib.dsa_mla_workspace_size(64, 128, 512, 2048) == 0
+    assert lib.dsa_mla_workspace_size(2, 128, 512, 100) == 0   # two tiles per query: no split
+    assert lib.dsa_mla_workspace_size(0, 128, 512, 2048) == 0
+    assert lib.dsa_mla_workspace_size(4, 64, 512, 2048) == 0    # not the tensor-core shape
