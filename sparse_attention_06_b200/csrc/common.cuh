@@ -157,12 +157,6 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
-// 16-byte cp.async (L2 only); src_bytes < 16 zero-fills the rest of the destination.
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-
 // 4-byte cp.async (through L1), for scattered scalars.
 __device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
@@ -205,32 +199,12 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16/f16 inputs, f32 accumulate).
-__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16: A (M rows x 16 K) read from tensor memory,
-// one row per lane, two consecutive K elements per 32-bit column.
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Issue-lean forms for unrolled MMA chains: the accumulate flag is a compile-time constant and
-// there is no memory clobber (ordering against shared-memory writes comes from the fences and
-// mbarrier waits around the chain, which are volatile asm with clobbers themselves).
+// D[tmem] (+)= A * B^T, kind::f16 (bf16/f16 inputs, f32 accumulate): umma_ss with A and B from
+// shared-memory descriptors, umma_ts with A (M rows x 16 K) read from tensor memory, one row per
+// lane, two consecutive K elements per 32-bit column.  Issue-lean forms for unrolled chains: the
+// accumulate flag is a compile-time constant and there is no memory clobber (ordering against
+// shared-memory writes comes from the fences and mbarrier waits around the chain, which are
+// volatile asm with clobbers themselves).
 template <int ACC>
 __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc) {
   asm volatile(
