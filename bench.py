@@ -5,8 +5,10 @@
 One step is one pass of the whole hot path over one batch of synthetic, seeded input: indexer
 scores (dsa_indexer_scores), top-K selection (dsa_topk_select) and sparse MLA
 (dsa_sparse_mla_decode, or dsa_sparse_mla_prefill for the prefill chunk).  The default workload
-is bf16 decode at batch 1, context 32768 (indexer 64 heads x 128, top-2048, MLA 128 heads over
-512 + 64).  Other workloads: tiny, batched_decode, prefill, long_decode (see dsa_inputs.py).
+is batched bf16 decode: 64 requests with context lengths uniform in [4096, 131072], paged in
+64-token blocks with shuffled block tables (indexer 64 heads x 128, top-2048, MLA 128 heads over
+512 + 64) -- the largest single-GPU workload by bytes.  Other workloads: tiny, decode (batch 1,
+context 32768), prefill, long_decode (see dsa_inputs.py).
 
 Timing: W untimed warm-up steps; then K steps, each bracketed by CUDA events on the launching
 stream; when one copy of the workload's resident data fits in L2, the steps rotate over enough
@@ -24,6 +26,7 @@ import argparse
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -75,11 +78,18 @@ def work_model(spec):
     sel = [min(v, spec.k) for v in vis]
     topk_bytes = pairs * 4 + T * spec.k * 4
     mla_rows = sum(sel)
-    mla_bytes = mla_rows * spec.dqk * act + T * spec.H * (spec.dqk + spec.d_v) * act + T * spec.H * 4
+    # HBM bytes of the row gather: a row that several queries of one request select is read from
+    # HBM once at best (the others hit L2), so a request costs at most its visible rows
+    sel_req = {}
+    for t in range(T):
+        r = spec.q_req[t]
+        sel_req[r] = sel_req.get(r, 0) + sel[t]
+    mla_hbm_rows = sum(min(sel_req[r], per_req[r]) for r in sel_req)
+    mla_bytes = mla_hbm_rows * spec.dqk * act + T * spec.H * (spec.dqk + spec.d_v) * act + T * spec.H * 4
     mla_flops = 2.0 * spec.H * mla_rows * (spec.dqk + spec.d_v)
     return dict(indexer_bytes=idx_bytes, indexer_flops=idx_flops, topk_bytes=topk_bytes,
                 mla_bytes=mla_bytes, mla_flops=mla_flops, key_tokens=key_tokens, pairs=pairs,
-                mla_rows=mla_rows)
+                mla_rows=mla_rows, mla_hbm_rows=mla_hbm_rows)
 
 
 def resident_bytes(spec, x):
@@ -100,9 +110,19 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+def source_digest(path):
+    """First 16 hex digits of the sha256 of a source file's code with comments and runs of white
+    space removed: edits of comments alone keep the digest, any change of code changes it."""
+    import hashlib
+    src = open(path).read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return hashlib.sha256(" ".join(src.split()).encode()).hexdigest()[:16]
+
+
 def ncu_traffic(kernel, workload):
     """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None when there is
-    none for this kernel and workload, or when the kernel's source changed since the capture."""
+    none for this kernel and workload, or when the kernel's code changed since the capture."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -111,10 +131,7 @@ def ncu_traffic(kernel, workload):
         e = d.get("%s@%s" % (kernel, workload))
         if not e:
             return None
-        src = os.path.join(ROOT, e["source"])
-        import hashlib
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        if h != e["source_sha"]:
+        if source_digest(os.path.join(ROOT, e["source"])) != e["source_digest"]:
             return None
         return float(e["bytes_per_launch"])
     except Exception:
@@ -441,7 +458,7 @@ def cpu_baseline(x, spec, budget_s=15.0, repeats=None):
     budget_pairs = max(1, int(budget_s * cores * 1e8 / (spec.Hi * spec.Di + 1)))
     qs = _sample_queries(spec, budget_pairs)
     sub = di.subset(x, qs)
-    threads = min(cores, len(qs))
+    threads = cores
     t0 = time.perf_counter()
     n = 0
     while True:
@@ -475,7 +492,7 @@ def run_reference(args):
     budget_pairs = max(1, int(budget * cores * 1e8 / (spec.Hi * spec.Di + 1)))
     qs = _sample_queries(spec, budget_pairs)
     sub = di.subset(x, qs)
-    threads = min(cores, len(qs))
+    threads = cores
     for _ in range(args.warmup):
         oracle_step(sub, spec, threads)
     t0 = time.perf_counter()
@@ -502,7 +519,7 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="decode",
+    ap.add_argument("--config", default="batched_decode",
                     choices=["tiny", "decode", "batched_decode", "prefill", "long_decode", "profile_decode",
                              "profile_prefill", "profile_long"])
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])

@@ -177,12 +177,17 @@ dsa_status dsa_sparse_mla_prefill(const void* q, int32_t q_dtype, int32_t H, int
  * convenience entry point for callers that cannot allocate device memory (for example code that
  * runs inside another framework's memory pool, or on a path where allocation is not allowed).
  * Same inputs, outputs and results as dsa_sparse_mla_decode; the split partials go to a fixed
- * 32 MiB scratch array inside the library (held on every GPU that loads the library until the
- * process exits).  Sizes whose partials need more than that return DSA_ERR_INVALID_ARG with a
- * message (use dsa_sparse_mla_decode with a workspace then).  Allocates nothing.
- * The first call on each device looks up the scratch address (cudaGetSymbolAddress); make that
- * first call before any stream capture.  All calls share the scratch: calls whose kernels overlap
- * on the GPU race; calls ordered on one stream are safe.  Nothing in the scratch needs clearing.
+ * 32 MiB scratch array inside the library.  Calls whose partials need more than that (the same
+ * split plan as dsa_sparse_mla_decode; shapes that take the generic kernels need none) return
+ * DSA_ERR_INVALID_ARG with a message: use dsa_sparse_mla_decode with a workspace then.
+ * Set-up: the first call on each device looks up the scratch address (cudaGetSymbolAddress).
+ * Under lazy module loading, the CUDA default, that lookup is when the scratch is reserved on the
+ * device (32 MiB, held until the process exits), and it may synchronise the device.  Make the
+ * first call on each device during set-up, before timing-critical work and before any stream
+ * capture; later calls allocate nothing and do not synchronise.  After a device reset the next
+ * call looks the address up again.  All calls on a device share the scratch: calls whose kernels
+ * overlap on the GPU race; calls ordered on one stream are safe.  Nothing in the scratch needs
+ * clearing.
  */
 dsa_status dsa_sparse_mla_decode_noalloc(const void* q, int32_t q_dtype, int32_t H, int32_t d_v,
                                          int32_t d_rope, const dsa_paged_cache* latent,
@@ -192,6 +197,13 @@ dsa_status dsa_sparse_mla_decode_noalloc(const void* q, int32_t q_dtype, int32_t
 
 /* Bytes of workspace dsa_sparse_mla_decode needs for these sizes (0 when none). Host only. */
 size_t dsa_mla_workspace_size(int32_t num_queries, int32_t H, int32_t d_v, int32_t k);
+
+/* Diagnostic of the bounded waits (no counterpart on the pages): enqueues one kernel whose single
+ * thread waits on an mbarrier phase that never completes, with the same bounded wait the
+ * tensor-core kernels use but a limit of `limit_cycles` SM cycles (1 .. 4e9).  The wait gives up,
+ * the kernel sets DSA_DEVERR_TIMEOUT in the device error word and returns; the context stays
+ * usable.  Read the word with dsa_get_device_error. */
+dsa_status dsa_selftest_bounded_wait(int64_t limit_cycles, dsa_stream stream);
 
 /* Synchronises `stream`, then reads the device error word of the current device into *code
  * (0 = no fault).  Not for use inside stream capture. */

@@ -4,7 +4,7 @@ TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the 
 ``cpu_baseline`` leg (and its ``--impl reference`` arm) may import this package.  It shares no
 code with the CUDA path in ``sparse_attention_06_b200`` and imports nothing from it.
 
-The arithmetic lives in ``dsa_oracle.c`` (plain C, double precision, OpenMP over queries); this
+The arithmetic lives in ``dsa_oracle.c`` (plain C, double precision, OpenMP over independent key positions, queries and heads); this
 module only compiles it with gcc and marshals numpy / torch CPU arrays into it.  Every function
 states the passage it follows in the C source.  Pins of the oracle against values fixed by the
 pages and by mathematics are in ``tests/test_oracle_pins.py``.

@@ -26,7 +26,8 @@
  *   - LSE is the natural-log log-sum-exp of the scaled logits.
  *
  * Everything is computed in double from the same quantised inputs the GPU sees.  Loops follow
- * the definitions one-to-one; the only parallelism is OpenMP over independent queries.
+ * the definitions one-to-one; the only parallelism is OpenMP over independent items: the key
+ * positions of a query (indexer), the queries (selection) and the heads of a query (attention).
  * The paged address rule (logical position -> physical row) is the plain one:
  *   row = block_table[req][pos / block_size] * block_size + pos % block_size.
  */
@@ -109,28 +110,32 @@ void oracle_indexer_scores(int T, const void* q, int q_dtype, int Hi, int Di, co
                            const int32_t* block_table, int max_blocks, const int32_t* q_req,
                            const int32_t* q_pos, double* out, int64_t ld, int nthreads) {
   set_threads(nthreads);
-#pragma omp parallel for schedule(dynamic, 1)
+  double* qt = (double*)malloc(sizeof(double) * (size_t)Hi * (size_t)Di);
   for (int t = 0; t < T; ++t) {
-    double* khat = (double*)malloc(sizeof(double) * (size_t)Di);
-    double* qt = (double*)malloc(sizeof(double) * (size_t)Hi * (size_t)Di);
     for (int64_t e = 0; e < (int64_t)Hi * Di; ++e) qt[e] = load_elem(q, q_dtype, (int64_t)t * Hi * Di + e);
     int64_t n = (int64_t)q_pos[t] + 1;
-    for (int64_t s = 0; s < n; ++s) {
-      int64_t row = physical_row(block_table, max_blocks, block_size, q_req[t], s);
-      double sc = (k_dtype == OR_E4M3) ? (double)key_scale[row] : 1.0;
-      for (int i = 0; i < Di; ++i) khat[i] = load_elem(kpool, k_dtype, row * Di + i) * sc;
-      double score = 0.0;
-      for (int h = 0; h < Hi; ++h) {
-        double dot = 0.0;
-        for (int i = 0; i < Di; ++i) dot += qt[(int64_t)h * Di + i] * khat[i];
-        double relu = dot > 0.0 ? dot : 0.0;
-        score += (double)w[(int64_t)t * Hi + h] * relu;
+    /* the key positions of one query are independent: they are shared out among the threads */
+#pragma omp parallel
+    {
+      double* khat = (double*)malloc(sizeof(double) * (size_t)Di);
+#pragma omp for schedule(static)
+      for (int64_t s = 0; s < n; ++s) {
+        int64_t row = physical_row(block_table, max_blocks, block_size, q_req[t], s);
+        double sc = (k_dtype == OR_E4M3) ? (double)key_scale[row] : 1.0;
+        for (int i = 0; i < Di; ++i) khat[i] = load_elem(kpool, k_dtype, row * Di + i) * sc;
+        double score = 0.0;
+        for (int h = 0; h < Hi; ++h) {
+          double dot = 0.0;
+          for (int i = 0; i < Di; ++i) dot += qt[(int64_t)h * Di + i] * khat[i];
+          double relu = dot > 0.0 ? dot : 0.0;
+          score += (double)w[(int64_t)t * Hi + h] * relu;
+        }
+        out[(int64_t)t * ld + s] = score;
       }
-      out[(int64_t)t * ld + s] = score;
+      free(khat);
     }
-    free(khat);
-    free(qt);
   }
+  free(qt);
 }
 
 /* Order used by the selection: higher score first; equal scores -> lower position first. */
@@ -196,47 +201,51 @@ void oracle_sparse_mla(int T, const void* q, int q_dtype, int H, int Dqk, int Dv
                        int max_blocks, const int32_t* q_req, const int32_t* idx, int K,
                        double scale, double* out, double* lse, int nthreads) {
   set_threads(nthreads);
-#pragma omp parallel for schedule(dynamic, 1)
+  int64_t* rows = (int64_t*)malloc(sizeof(int64_t) * (size_t)K);
+  double* lat = (double*)malloc(sizeof(double) * (size_t)K * (size_t)Dqk);
   for (int t = 0; t < T; ++t) {
     int nsel = 0;
-    int64_t* rows = (int64_t*)malloc(sizeof(int64_t) * (size_t)K);
     for (int j = 0; j < K; ++j) {
       int32_t p = idx[(int64_t)t * K + j];
       if (p >= 0) rows[nsel++] = physical_row(block_table, max_blocks, block_size, q_req[t], p);
     }
-    double* lat = (double*)malloc(sizeof(double) * (size_t)(nsel > 0 ? nsel : 1) * (size_t)Dqk);
     for (int j = 0; j < nsel; ++j)
       for (int i = 0; i < Dqk; ++i) lat[(int64_t)j * Dqk + i] = load_elem(lpool, l_dtype, rows[j] * Dqk + i);
-    double* logit = (double*)malloc(sizeof(double) * (size_t)(nsel > 0 ? nsel : 1));
-    double* qh = (double*)malloc(sizeof(double) * (size_t)Dqk);
-    for (int h = 0; h < H; ++h) {
-      double* o = out + ((int64_t)t * H + h) * Dv;
-      for (int i = 0; i < Dqk; ++i) qh[i] = load_elem(q, q_dtype, ((int64_t)t * H + h) * Dqk + i);
-      if (nsel == 0) {
+    /* the heads of one query are independent: they are shared out among the threads */
+#pragma omp parallel
+    {
+      double* logit = (double*)malloc(sizeof(double) * (size_t)(nsel > 0 ? nsel : 1));
+      double* qh = (double*)malloc(sizeof(double) * (size_t)Dqk);
+#pragma omp for schedule(static)
+      for (int h = 0; h < H; ++h) {
+        double* o = out + ((int64_t)t * H + h) * Dv;
+        for (int i = 0; i < Dqk; ++i) qh[i] = load_elem(q, q_dtype, ((int64_t)t * H + h) * Dqk + i);
+        if (nsel == 0) {
+          for (int c = 0; c < Dv; ++c) o[c] = 0.0;
+          if (lse) lse[(int64_t)t * H + h] = -INFINITY;
+          continue;
+        }
+        double m = -INFINITY;
+        for (int j = 0; j < nsel; ++j) {
+          double dot = 0.0;
+          for (int i = 0; i < Dqk; ++i) dot += qh[i] * lat[(int64_t)j * Dqk + i];
+          logit[j] = scale * dot;
+          if (logit[j] > m) m = logit[j];
+        }
+        double z = 0.0;
         for (int c = 0; c < Dv; ++c) o[c] = 0.0;
-        if (lse) lse[(int64_t)t * H + h] = -INFINITY;
-        continue;
+        for (int j = 0; j < nsel; ++j) {
+          double p = exp(logit[j] - m);
+          z += p;
+          for (int c = 0; c < Dv; ++c) o[c] += p * lat[(int64_t)j * Dqk + c];
+        }
+        for (int c = 0; c < Dv; ++c) o[c] /= z;
+        if (lse) lse[(int64_t)t * H + h] = m + log(z);
       }
-      double m = -INFINITY;
-      for (int j = 0; j < nsel; ++j) {
-        double dot = 0.0;
-        for (int i = 0; i < Dqk; ++i) dot += qh[i] * lat[(int64_t)j * Dqk + i];
-        logit[j] = scale * dot;
-        if (logit[j] > m) m = logit[j];
-      }
-      double z = 0.0;
-      for (int c = 0; c < Dv; ++c) o[c] = 0.0;
-      for (int j = 0; j < nsel; ++j) {
-        double p = exp(logit[j] - m);
-        z += p;
-        for (int c = 0; c < Dv; ++c) o[c] += p * lat[(int64_t)j * Dqk + c];
-      }
-      for (int c = 0; c < Dv; ++c) o[c] /= z;
-      if (lse) lse[(int64_t)t * H + h] = m + log(z);
+      free(qh);
+      free(logit);
     }
-    free(qh);
-    free(logit);
-    free(lat);
-    free(rows);
   }
+  free(lat);
+  free(rows);
 }

@@ -34,7 +34,7 @@ EXPORTED = (
     "dsa_indexer_scores", "dsa_topk_select", "dsa_indexer_topk", "dsa_sparse_mla_decode",
     "dsa_sparse_mla_prefill", "dsa_mla_workspace_size", "dsa_get_device_error",
     "dsa_clear_device_error", "dsa_status_string", "dsa_last_error_message", "dsa_abi_version",
-    "dsa_kernel_launch_count", "dsa_sparse_mla_decode_noalloc",
+    "dsa_kernel_launch_count", "dsa_sparse_mla_decode_noalloc", "dsa_selftest_bounded_wait",
 )
 
 
@@ -85,6 +85,7 @@ def load_library():
         "dsa_sparse_mla_decode_noalloc": [P, I32, I32, I32, I32, PC, PB, P, I32, F, P, P, P],
         "dsa_get_device_error": [ctypes.POINTER(I32), P],
         "dsa_clear_device_error": [P],
+        "dsa_selftest_bounded_wait": [I64, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -251,6 +252,12 @@ def dsa_get_device_error(stream=None) -> int:
 def dsa_kernel_launch_count() -> int:
     """Kernels the library has enqueued in this process so far."""
     return int(load_library().dsa_kernel_launch_count())
+
+
+def dsa_selftest_bounded_wait(limit_cycles, stream=None):
+    """Diagnostic: a kernel whose bounded wait on a phase that never completes gives up after
+    ``limit_cycles`` SM cycles and sets DEVERR_TIMEOUT (include/dsa.h)."""
+    _check(load_library().dsa_selftest_bounded_wait(int(limit_cycles), _stream(stream)))
 
 
 def dsa_clear_device_error(stream=None):

@@ -79,21 +79,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Number of try_wait rounds before a wait is declared lost.  Each try_wait may suspend the
-// thread for a hardware-chosen interval; with the clock check below the wait gives up after
-// roughly kWaitCycles SM cycles (about two seconds at 1.9 GHz).
+// Default limit of a bounded wait, in SM cycles (about two seconds at 1.9 GHz); a wait that has
+// not seen its phase complete by then gives up.
 constexpr long long kWaitCycles = 4000000000LL;
 
 // Bounded wait on an mbarrier phase.  Returns false (and raises DSA_DEVERR_TIMEOUT) when the
-// phase did not complete in time or when another role of this CTA already gave up (*abort).
+// phase did not complete within `limit` SM cycles, or when another role of this CTA already gave
+// up (*abort_flag).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err,
-                                          volatile int* abort_flag) {
+                                          volatile int* abort_flag, long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort_flag && *abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       raise_error(err, DSA_DEVERR_TIMEOUT);
       if (abort_flag) *abort_flag = 1;
       return false;

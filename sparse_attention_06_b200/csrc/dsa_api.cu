@@ -18,33 +18,61 @@ namespace dsa {
 namespace {
 
 thread_local char g_msg[256];
+constexpr int kMaxDevices = 64;
 
 dsa_status fail(dsa_status st, const char* fmt, const char* detail = "") {
   snprintf(g_msg, sizeof g_msg, fmt, detail);
   return st;
 }
 
-constexpr int kMaxDevices = 64;
-int* g_err_ptr[kMaxDevices];
-int g_num_sms[kMaxDevices];
 std::mutex g_mu;
 std::atomic<long long> g_launches{0};
 
-// Device address of the error word and the SM count of the current device (looked up once).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The calling thread's current CUDA context (NULL when none is current yet).
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+  return c;
+}
+
+struct DeviceEntry {
+  CUcontext ctx;
+  int* err;
+  int num_sms;
+};
+DeviceEntry g_dev[kMaxDevices];
+
+// Device address of the error word and the SM count of the current device, looked up once per
+// device and looked up again whenever the device's context is not the one they were found in
+// (after a device reset the old addresses are gone).
 bool device_state(int** err, int* num_sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_err_ptr[dev]) {
+  DeviceEntry& d = g_dev[dev];
+  CUcontext ctx = current_context();
+  if (!d.err || !ctx || ctx != d.ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_dsa_device_error) != cudaSuccess) return false;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
-    g_num_sms[dev] = sms;
-    g_err_ptr[dev] = static_cast<int*>(p);
+    d.num_sms = sms;
+    d.err = static_cast<int*>(p);
+    d.ctx = current_context();
   }
-  *err = g_err_ptr[dev];
-  *num_sms = g_num_sms[dev];
+  *err = d.err;
+  *num_sms = d.num_sms;
   return true;
 }
 
@@ -111,6 +139,25 @@ EncodeTiledFn encode_fn() {
 }  // namespace
 
 void set_last_error_message(const char* msg) { snprintf(g_msg, sizeof g_msg, "%s", msg); }
+
+CUcontext current_cuda_context() { return current_context(); }
+
+bool current_device_sms(int* num_sms) {
+  int* err;
+  return device_state(&err, num_sms);
+}
+
+MlaPlan mla_plan(bool decode, const void* q, int32_t q_dtype, int32_t H, int32_t d_v, int32_t d_rope,
+                 const dsa_paged_cache& latent, int32_t T, int32_t k, const void* out, int num_sms) {
+  MlaPlan pl{false, 1, 0};
+  pl.tensor_cores = H == 128 && d_v == 512 && d_rope == 64 && q_dtype == DSA_BF16 && latent.block_size == 64 &&
+                    aligned16(q) && aligned16(out) && aligned16(latent.data);
+  if (pl.tensor_cores && T > 0) {
+    pl.nsplit = decode ? mla_tc_num_splits(T, k, num_sms) : 1;
+    pl.workspace_bytes = mla_tc_workspace_bytes(T, H, d_v, pl.nsplit);
+  }
+  return pl;
+}
 
 bool encode_tmap_2d(void* tmap_out, const void* base, int elem_bytes, uint64_t inner,
                     uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
@@ -255,19 +302,16 @@ static dsa_status mla_common(bool decode, const void* q, int32_t q_dtype, int32_
   if (!device_state(&err, &sms)) return fail(DSA_ERR_CUDA, "no CUDA device%s");
   MlaArgs a{q, q_dtype, H, d_v, d_rope, *latent, *batch, idx, k, softmax_scale, out, lse,
             workspace, workspace_bytes, err};
-  const bool tc_shape = H == 128 && d_v == 512 && d_rope == 64 && q_dtype == DSA_BF16 &&
-                        latent->block_size == 64 && aligned16(q) && aligned16(out) &&
-                        aligned16(latent->data);
+  const int T = batch->num_queries;
+  const MlaPlan pl = mla_plan(decode, q, q_dtype, H, d_v, d_rope, *latent, T, k, out, sms);
   cudaError_t e;
   int kernels = 1;
-  if (tc_shape) {
-    const int T = batch->num_queries;
-    const int nsplit = decode ? mla_tc_num_splits(T, k, sms) : 1;
-    const size_t need = mla_tc_workspace_bytes(T, H, d_v, nsplit);
+  if (pl.tensor_cores) {
+    const size_t need = pl.workspace_bytes;
     if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)))
       return fail(DSA_ERR_INVALID_ARG, "mla: workspace missing, too small or not 256-byte aligned%s");
-    kernels = nsplit > 1 ? 2 : 1;
-    e = launch_mla_tc(a, nsplit, sms, static_cast<cudaStream_t>(stream));
+    kernels = pl.nsplit > 1 ? 2 : 1;
+    e = launch_mla_tc(a, pl.nsplit, sms, static_cast<cudaStream_t>(stream));
   } else {
     e = launch_mla_generic(a, static_cast<cudaStream_t>(stream));
   }
@@ -291,6 +335,16 @@ dsa_status dsa_sparse_mla_prefill(const void* q, int32_t q_dtype, int32_t H, int
                                   size_t workspace_bytes, dsa_stream stream) {
   return mla_common(false, q, q_dtype, H, d_v, d_rope, latent, batch, idx, k, softmax_scale, out,
                     lse, workspace, workspace_bytes, stream);
+}
+
+dsa_status dsa_selftest_bounded_wait(int64_t limit_cycles, dsa_stream stream) {
+  if (limit_cycles < 1 || limit_cycles > kWaitCycles)
+    return fail(DSA_ERR_INVALID_ARG, "selftest: limit_cycles must be in [1, 4e9]%s");
+  int* err;
+  int sms;
+  if (!device_state(&err, &sms)) return fail(DSA_ERR_CUDA, "no CUDA device%s");
+  return cuda_status(launch_bounded_wait_selftest(limit_cycles, err, static_cast<cudaStream_t>(stream)),
+                     "dsa_selftest_bounded_wait launch", 1);
 }
 
 size_t dsa_mla_workspace_size(int32_t num_queries, int32_t H, int32_t d_v, int32_t k) {

@@ -1,6 +1,7 @@
 // internal.h -- launchers shared between the C-ABI layer and the kernel files.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -80,6 +81,25 @@ inline cudaLaunchConfig_t launch_config(dim3 grid, dim3 block, size_t smem, cuda
 
 // detail text returned by dsa_last_error_message() on this host thread
 void set_last_error_message(const char* msg);
+
+// the calling thread's current CUDA context (NULL when none is current)
+CUcontext current_cuda_context();
+
+// SM count of the current device (false when there is no usable device)
+bool current_device_sms(int* num_sms);
+
+// How an MLA call runs: on the tensor-core kernels or the generic ones, with how many key splits
+// per query, and the workspace bytes of the split partials (0 with one split or the generic path).
+struct MlaPlan {
+  bool tensor_cores;
+  int nsplit;
+  size_t workspace_bytes;
+};
+MlaPlan mla_plan(bool decode, const void* q, int32_t q_dtype, int32_t H, int32_t d_v, int32_t d_rope,
+                 const dsa_paged_cache& latent, int32_t T, int32_t k, const void* out, int num_sms);
+
+// diagnostic: one thread waits on an mbarrier that nothing arrives on, bounded by limit_cycles
+cudaError_t launch_bounded_wait_selftest(long long limit_cycles, int* err, cudaStream_t s);
 
 // tensor-map encoding through the driver entry point (no link-time libcuda dependency)
 bool encode_tmap_2d(void* tmap_out, const void* base, int elem_bytes, uint64_t inner,

@@ -60,13 +60,20 @@ def run_gpu(x, mla_entry="decode"):
     return dict(scores=scores, idx=idx, out=out, lse=lse, err=err)
 
 
-def parity_case(x, queries=None, kind="bf16", mla_entry="decode", e2e_min_overlap=0.999):
+def parity_case(x, queries=None, kind="bf16", mla_entry="decode", e2e_min_overlap=0.999, topk_all_rows=False):
     """Full parity of one workload ``x`` (tensors on cuda): GPU path vs the oracle on the queries
-    listed (all by default).  Returns a dict of the measured errors."""
+    listed (all by default).  With ``topk_all_rows`` the selection of every query (not only the
+    listed ones) is checked bit-exactly against the oracle's selection from the GPU's own scores.
+    Returns a dict of the measured errors."""
     spec = x["spec"]
     tol = TOL[kind]
     g = run_gpu(x, mla_entry)
     assert g["err"] == 0, "device error word %d" % g["err"]
+    if topk_all_rows:
+        qpos_all = x["q_pos"].cpu().numpy()
+        for r0 in range(0, spec.T, 64):  # rows in chunks: the f64 copy of all scores can be GBs
+            r1 = min(spec.T, r0 + 64)
+            check_topk(g["idx"][r0:r1].cpu(), g["scores"][r0:r1].cpu(), qpos_all[r0:r1], spec.k)
     qs = list(range(spec.T)) if queries is None else list(queries)
     sub = subset_cpu(x, qs)
     qpos = sub["q_pos"].numpy()

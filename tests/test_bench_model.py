@@ -34,3 +34,14 @@ def test_work_model_prefill_pairs():
     m = bench.work_model(spec)
     assert m["pairs"] == sum(65537 + t for t in range(4096))
     assert m["indexer_flops"] == pytest.approx(4.54e12, rel=0.01)
+
+
+def test_work_model_prefill_row_gather_hbm_bytes():
+    # the 4096 queries of the prefill chunk select 4096 x 2048 rows, but they all come from one
+    # request of 69632 positions: HBM serves each row at most once
+    spec = di.prefill()
+    m = bench.work_model(spec)
+    assert m["mla_rows"] == 4096 * 2048
+    assert m["mla_hbm_rows"] == 65536 + 4096
+    dec = bench.work_model(di.batched_decode())
+    assert dec["mla_hbm_rows"] == dec["mla_rows"] == 64 * 2048

@@ -1,7 +1,9 @@
 """Parity at the full sizes of the five workloads, in the launch configuration the benchmark
 times: the whole hot path runs on the GPU for every query; the fp64 oracle recomputes sampled
 queries one by one (all scores of the sampled query, its selection from the GPU's scores, and its
-attention output) and the end-to-end selection from the oracle's own scores must agree."""
+attention output) and the end-to-end selection from the oracle's own scores must agree.  The
+selection of every query of every workload is checked bit-exactly against the oracle's selection
+applied to the GPU's own scores."""
 import gc
 
 import pytest
@@ -24,7 +26,7 @@ def test_fullsize_sampled(name, queries, kind, entry):
     spec = di.WORKLOADS[name]()
     x = di.generate(spec, "cuda")
     try:
-        r = parity_case(x, queries=queries, kind=kind, mla_entry=entry)
+        r = parity_case(x, queries=queries, kind=kind, mla_entry=entry, topk_all_rows=True)
         print(name, r)
     finally:
         del x

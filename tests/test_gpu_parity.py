@@ -250,3 +250,20 @@ def test_bad_block_id_and_bad_index_flagged():
     assert torch.allclose(out[0].float(), row.expand(spec.H, -1), atol=1e-2)
     dsa.dsa_clear_device_error()
     assert dsa.dsa_get_device_error() == 0
+
+
+# ---------------------------------------------------------------------------------------------
+# bounded waits: a wait that runs out sets the timeout bit and the kernel returns
+# ---------------------------------------------------------------------------------------------
+
+def test_bounded_wait_runs_out_and_context_stays_usable():
+    dsa.dsa_clear_device_error()
+    dsa.dsa_selftest_bounded_wait(2_000_000)  # about 1 ms of SM cycles; nothing completes the phase
+    err = dsa.dsa_get_device_error()
+    assert err & dsa.DEVERR_TIMEOUT
+    dsa.dsa_clear_device_error()
+    assert dsa.dsa_get_device_error() == 0
+    # the context is still usable: a small layer passes parity afterwards
+    spec = _spec([2300], seed=33)
+    x = to_dev(di.generate(spec, "cpu"))
+    parity_case(x, kind="bf16")

@@ -66,3 +66,22 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     with pytest.raises(dsa.DsaError) as e:
         dsa.dsa_sparse_mla_decode_noalloc(x["q_mla"], lat, batch, idx, spec.scale, out)
     assert e.value.status == dsa.DSA_ERR_INVALID_ARG and "scratch" in str(e.value)
+
+
+def test_noalloc_generic_shape_needs_no_scratch():
+    # f32 operands take the generic kernels, which use no split partials: a batch whose bf16
+    # tensor-core plan would exceed the scratch is accepted and matches the workspace entry point
+    T = next((t for t in range(2, 1024) if dsa.dsa_mla_workspace_size(t, 128, 512, 2048) > 32 << 20), None)
+    spec = di.Spec("noalloc_f32", lens=[2100] * T, q_req=list(range(T)), q_pos=[2099] * T, act_dtype="f32",
+                   key_dtype="f32", seed=43)
+    x = to_dev(di.generate(spec, "cpu"))
+    keys, lat, batch, max_ctx = cache_and_batch(x)
+    idx = torch.empty((spec.T, spec.k), dtype=torch.int32, device="cuda")
+    scores = torch.empty((spec.T, (max_ctx + 3) // 4 * 4), dtype=torch.float32, device="cuda")
+    dsa.dsa_indexer_topk(x["q_idx"], x["w"], keys, batch, spec.k, scores, idx)
+    ref = torch.empty((spec.T, spec.H, spec.d_v), dtype=torch.float32, device="cuda")
+    dsa.dsa_sparse_mla_decode(x["q_mla"], lat, batch, idx, spec.scale, ref)
+    out = torch.full_like(ref, float("nan"))
+    dsa.dsa_sparse_mla_decode_noalloc(x["q_mla"], lat, batch, idx, spec.scale, out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
