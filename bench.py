@@ -87,6 +87,12 @@ def work_model(spec):
     mla_hbm_rows = sum(min(sel_req[r], per_req[r]) for r in sel_req)
     mla_bytes = mla_hbm_rows * spec.dqk * act + T * spec.H * (spec.dqk + spec.d_v) * act + T * spec.H * 4
     mla_flops = 2.0 * spec.H * mla_rows * (spec.dqk + spec.d_v)
+    if max(vis) <= spec.k:
+        # the dense case: every query keeps all its positions, no indexer or selection runs
+        idx_bytes = idx_flops = topk_bytes = 0
+    # IndexShare: the group's other layers run sparse MLA on the same selection
+    mla_bytes *= spec.share_layers
+    mla_flops *= spec.share_layers
     return dict(indexer_bytes=idx_bytes, indexer_flops=idx_flops, topk_bytes=topk_bytes,
                 mla_bytes=mla_bytes, mla_flops=mla_flops, key_tokens=key_tokens, pairs=pairs,
                 mla_rows=mla_rows, mla_hbm_rows=mla_hbm_rows)
@@ -246,8 +252,21 @@ class Layer:
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev) if ws else None
         self.prefill = spec.query_group > 1
         self.q_idx, self.w, self.q_mla = x["q_idx"], x["w"], x["q_mla"]
+        # every query sees at most K positions: the method keeps them all, so the layer is
+        # attention over the whole context without indexer or selection (the dense case)
+        self.dense = self.max_ctx <= spec.k
+        # IndexShare: layers that reuse this layer's selection (own MLA queries and latent cache)
+        self.shared = []
+        for sh in x.get("shared", []):
+            self.shared.append((sh["q_mla"], dsa.PagedCache(sh["latent_pool"]), torch.empty_like(self.out),
+                                torch.empty_like(self.lse)))
 
-    def step(self, ev=None):
+    def _mla(self, q, lat, out, lse, idx):
+        fn = self.dsa.dsa_sparse_mla_prefill if self.prefill else self.dsa.dsa_sparse_mla_decode
+        fn(q, lat, self.batch, idx, self.spec.scale, out, lse, self.ws, k=self.spec.k)
+
+    def step_sparse(self, ev=None):
+        """Indexer -> top-K -> sparse MLA (and the shared layers' sparse MLA on the same selection)."""
         d = self.dsa
         d.dsa_indexer_scores(self.q_idx, self.w, self.keys, self.batch, self.scores)
         if ev is not None:
@@ -255,8 +274,39 @@ class Layer:
         d.dsa_topk_select(self.scores, self.batch.q_pos, self.spec.k, self.idx)
         if ev is not None:
             ev[1].record()
-        fn = d.dsa_sparse_mla_prefill if self.prefill else d.dsa_sparse_mla_decode
-        fn(self.q_mla, self.lat, self.batch, self.idx, self.spec.scale, self.out, self.lse, self.ws)
+        self._mla(self.q_mla, self.lat, self.out, self.lse, self.idx)
+        for q, lat, out, lse in self.shared:
+            self._mla(q, lat, out, lse, self.idx)
+
+    def step(self, ev=None):
+        if not self.dense:
+            return self.step_sparse(ev)
+        if ev is not None:
+            ev[0].record()
+            ev[1].record()
+        self._mla(self.q_mla, self.lat, self.out, self.lse, None)
+
+    def step_full_layer(self):
+        """One full layer alone (indexer, top-K, sparse MLA): the IndexShare comparison."""
+        d = self.dsa
+        d.dsa_indexer_scores(self.q_idx, self.w, self.keys, self.batch, self.scores)
+        d.dsa_topk_select(self.scores, self.batch.q_pos, self.spec.k, self.idx)
+        self._mla(self.q_mla, self.lat, self.out, self.lse, self.idx)
+
+
+def _time_steps(fn, K, stream):
+    """Device time of K back-to-back calls of fn, after a stream gate (CUDA events, ms)."""
+    import torch
+    b = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(GATE_CYCLES)
+    b.record(stream)
+    for i in range(K):
+        fn(i)
+    e.record(stream)
+    torch.cuda.synchronize()
+    return b.elapsed_time(e)
 
 
 def run_cuda(args):
@@ -276,8 +326,15 @@ def run_cuda(args):
     model = work_model(spec)
     # inputs larger than L2 between uses: rotate over identical copies of the resident data
     ncopy = max(1, -(-2 * L2_BYTES // max(1, resident_bytes(spec, x))))
-    copies = [x] + [{k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
-                    for _ in range(ncopy - 1)]
+    def clone(v):
+        if isinstance(v, torch.Tensor):
+            return v.clone()
+        if isinstance(v, list):
+            return [clone(e) for e in v]
+        if isinstance(v, dict):
+            return {k: clone(e) for k, e in v.items()}
+        return v
+    copies = [x] + [{k: clone(v) for k, v in x.items() if k != "spec"} | {"spec": spec} for _ in range(ncopy - 1)]
     layers = [Layer(c) for c in copies]
     layer = layers[0]
     stream = torch.cuda.current_stream()
@@ -333,10 +390,14 @@ def run_cuda(args):
 
     # end to end through the public API: per-step query-side inputs from pinned host memory,
     # the KV caches resident in HBM (state), output read back every step
-    names = ("q_idx", "w", "q_mla", "q_req", "q_pos", "block_table")
-    host_in = {n: x[n].cpu().pin_memory() for n in names}
+    names = ("q_req", "q_pos", "block_table", "q_mla") + (() if layer.dense else ("q_idx", "w"))
+
+    def query_inputs(c):  # device tensors of one copy that the host supplies every step
+        return [c[n] for n in names] + [sh["q_mla"] for sh in c.get("shared", [])]
+    host_in = [t.cpu().pin_memory() for t in query_inputs(x)]
+    dev_in = [query_inputs(c) for c in copies]
     host_out = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = host_out.numel() * host_out.element_size()
     e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     if world > 1:
@@ -346,15 +407,14 @@ def run_cuda(args):
         lay = layers[i % ncopy]
         torch.cuda.synchronize()  # end to end: every step starts from an idle device and host
         e2e_ev[i][0].record(stream)
-        for n, t in host_in.items():
-            lay.x[n].copy_(t, non_blocking=True)
+        for dst, src in zip(dev_in[i % ncopy], host_in):
+            dst.copy_(src, non_blocking=True)
         lay.step()
         host_out.copy_(lay.out, non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     e2e_s = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / 1e3, world, dev)
     e2e_value = aggregate(units, e2e_s, world)
-    err = dsa.dsa_get_device_error()
 
     # roofline of every kernel; the line's "roofline" is the dominant (slowest) one.  A kernel's
     # bound is whichever of its algorithmic bytes / HBM peak and FLOPs / tensor peak is larger.
@@ -364,6 +424,8 @@ def run_cuda(args):
     for name, ms_list, nbytes, flops in (("indexer", idx_ms, model["indexer_bytes"], model["indexer_flops"]),
                                          ("topk", topk_ms, model["topk_bytes"], 0.0),
                                          ("mla", mla_ms, model["mla_bytes"], model["mla_flops"])):
+        if nbytes == 0 and flops == 0:
+            continue  # not run in this workload (the dense case has no indexer or selection)
         t = statistics.mean(ms_list) / 1e3
         t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
         t_ten = flops / (tensor_peak * 1e12)
@@ -383,6 +445,21 @@ def run_cuda(args):
         breakdown[name + "_us"] = r["us"]
         breakdown[name + "_frac"] = r["frac"]
         breakdown[name + "_bound"] = r["bound"]
+
+    # comparisons on the same inputs: the sparse path where the dense case applies, and one full
+    # layer alone where a group of layers shares one selection
+    if layer.dense:
+        sp_ms = _time_steps(lambda i: layers[i % ncopy].step_sparse(), K, stream) / K
+        breakdown["sparse_path_us"] = sp_ms * 1e3
+        breakdown["dense_saving"] = 1.0 - ms_per_step / sp_ms
+    if layer.shared:
+        fl_ms = _time_steps(lambda i: layers[i % ncopy].step_full_layer(), K, stream) / K
+        n_l = 1 + len(layer.shared)
+        breakdown["layers_per_group"] = n_l
+        breakdown["full_layer_us"] = fl_ms * 1e3
+        breakdown["full_layers_us"] = n_l * fl_ms * 1e3
+        breakdown["group_saving"] = 1.0 - ms_per_step / (n_l * fl_ms)
+    err = dsa.dsa_get_device_error()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -424,27 +501,41 @@ def run_cuda(args):
 
 def oracle_step(sub, spec, nthreads):
     """One pass of the oracle over the queries in `sub` (indexer, selection, sparse MLA)."""
+    import numpy as np
     import oracle
-    s = oracle.indexer_scores(sub["q_idx"], sub["w"], sub["key_pool"], sub["key_scale"], sub["block_table"],
-                              sub["q_req"], sub["q_pos"], nthreads=nthreads)
-    idx = oracle.topk(s, sub["q_pos"], spec.k, nthreads=nthreads)
+    if int(sub["q_pos"].max()) + 1 <= spec.k:
+        # the dense case, as the layer runs it: every visible position, no indexer or selection
+        n = sub["q_pos"].numpy().astype(np.int64) + 1
+        j = np.arange(spec.k)[None, :]
+        idx = np.where(j < n[:, None], j, -1).astype(np.int32)
+    else:
+        s = oracle.indexer_scores(sub["q_idx"], sub["w"], sub["key_pool"], sub["key_scale"], sub["block_table"],
+                                  sub["q_req"], sub["q_pos"], nthreads=nthreads)
+        idx = oracle.topk(s, sub["q_pos"], spec.k, nthreads=nthreads)
     oracle.sparse_mla(sub["q_mla"], sub["latent_pool"], sub["block_table"], sub["q_req"], idx, spec.d_v,
                       spec.scale, nthreads=nthreads)
+    for sh in sub.get("shared", []):  # IndexShare: the other layers reuse the selection
+        oracle.sparse_mla(sh["q_mla"], sh["latent_pool"], sub["block_table"], sub["q_req"], idx, spec.d_v,
+                          spec.scale, nthreads=nthreads)
 
 
-def _sample_queries(spec, budget_pairs):
-    """Queries of a bounded sample: evenly spaced over the batch, up to `budget_pairs` visible
-    (query, key) pairs."""
+def oracle_macs(spec, t):
+    """Multiply-adds of one oracle pass over query t (indexer unless dense, attention per layer)."""
+    n = spec.q_pos[t] + 1
+    dense = max(spec.q_pos) + 1 <= spec.k
+    return (0 if dense else n * spec.Hi * spec.Di) + min(n, spec.k) * spec.H * (spec.dqk + spec.d_v) * spec.share_layers
+
+
+def _sample_queries(spec, budget_macs):
+    """Queries of a bounded sample: evenly spaced over the batch (at most 64), up to
+    `budget_macs` multiply-adds of oracle work."""
     T = spec.T
-    order = [int(round(i * (T - 1) / max(1, T - 1))) for i in range(T)]
-    if T > 1:
-        stride = max(1, T // 64)
-        order = list(range(0, T, stride))
-    qs, pairs = [], 0
+    order = list(range(0, T, max(1, T // 64)))
+    qs, macs = [], 0
     for t in order:
         qs.append(t)
-        pairs += spec.q_pos[t] + 1
-        if pairs >= budget_pairs:
+        macs += oracle_macs(spec, t)
+        if macs >= budget_macs:
             break
     return qs
 
@@ -454,9 +545,8 @@ def cpu_baseline(x, spec, budget_s=15.0, repeats=None):
     import dsa_inputs as di
     import oracle
     cores = oracle.max_threads()
-    # about 1e8 fp64 MAC/s per core in the indexer loop: size the sample to the budget
-    budget_pairs = max(1, int(budget_s * cores * 1e8 / (spec.Hi * spec.Di + 1)))
-    qs = _sample_queries(spec, budget_pairs)
+    # about 1e8 fp64 MAC/s per core in the oracle's loops: size the sample to the budget
+    qs = _sample_queries(spec, budget_s * cores * 1e8)
     sub = di.subset(x, qs)
     threads = cores
     t0 = time.perf_counter()
@@ -481,16 +571,13 @@ def run_reference(args):
     import torch
     import dsa_inputs as di
     spec = di.WORKLOADS[args.config]()
-    big = spec.name not in ("tiny_f32_L256",)
-    x = di.generate(spec, device="cpu") if not big or sum(spec.lens) <= 70000 else None
-    if x is None:
-        # draw the full workload only for the sampled queries' requests, on the CPU
-        x = di.generate(spec, device="cpu")
+    # the same seeded draw as the CUDA arm (on the GPU when there is one, else on the host); only
+    # the sampled queries' inputs go to the oracle
+    x = di.generate(spec, device="cuda" if torch.cuda.is_available() else "cpu")
     budget = min(args.cpu_budget, 120.0 / max(1, args.steps + args.warmup))
     import oracle
     cores = oracle.max_threads()
-    budget_pairs = max(1, int(budget * cores * 1e8 / (spec.Hi * spec.Di + 1)))
-    qs = _sample_queries(spec, budget_pairs)
+    qs = _sample_queries(spec, budget * cores * 1e8)
     sub = di.subset(x, qs)
     threads = cores
     for _ in range(args.warmup):
@@ -520,8 +607,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="batched_decode",
-                    choices=["tiny", "decode", "batched_decode", "prefill", "long_decode", "profile_decode",
-                             "profile_prefill", "profile_long"])
+                    choices=["tiny", "decode", "batched_decode", "prefill", "long_decode", "short_decode",
+                             "indexshare", "profile_decode", "profile_prefill", "profile_long"])
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -50,6 +50,7 @@ class Spec:
     planted_sigma: float = 0.0
     seed: int = 0x5EED
     query_group: int = 1       # queries come in runs of this many sharing one request
+    share_layers: int = 1      # layers in an IndexShare group: one full layer, the rest reuse its selection
 
     @property
     def T(self) -> int:
@@ -158,6 +159,12 @@ def generate(spec: Spec, device="cpu", with_mla=True, with_indexer=True):
     if with_mla:
         out["q_mla"] = normal((spec.T, spec.H, spec.dqk), act, dev, spec.seed, 4)
         out["latent_pool"] = normal((rows, spec.dqk), act, dev, spec.seed, 5).view(nblk, BLOCK, spec.dqk)
+        # IndexShare: the other layers of the group have their own MLA queries and latent caches
+        # (same requests, same paging) and no indexer inputs of their own
+        out["shared"] = [
+            {"q_mla": normal((spec.T, spec.H, spec.dqk), act, dev, spec.seed, 4 + 10 * l),
+             "latent_pool": normal((rows, spec.dqk), act, dev, spec.seed, 5 + 10 * l).view(nblk, BLOCK, spec.dqk)}
+            for l in range(1, spec.share_layers)]
     return out
 
 
@@ -231,6 +238,24 @@ def long_decode(B=16, L=202752, seed=0x5EED + 4) -> Spec:
                 q_pos=[L - 1] * B, key_dtype="e4m3", planted_frac=0.02, planted_sigma=3.0, seed=seed)
 
 
+def short_decode(B=64, lo=1024, hi=2048, seed=0x5EED + 8) -> Spec:
+    """bf16 batched decode at short contexts, uniform in [lo, hi] <= top-k: every query keeps all
+    of its positions (the dense case), so the layer is attention over the whole context."""
+    g = _gen("cpu", seed, 50)
+    lens = torch.randint(lo, hi + 1, (B,), generator=g).tolist()
+    return Spec("short_decode_bf16_B%d_L%d_%d" % (B, lo, hi), lens=lens, q_req=list(range(B)),
+                q_pos=[L - 1 for L in lens], seed=seed)
+
+
+def indexshare(B=64, lo=4096, hi=131072, layers=4, seed=0x5EED + 2) -> Spec:
+    """IndexShare group over the batched-decode workload: one full DSA layer (indexer, top-K,
+    sparse MLA) and ``layers - 1`` layers that reuse its selection (sparse MLA only)."""
+    s = batched_decode(B, lo, hi, seed)
+    s.name = "indexshare_x%d_batched_decode_bf16_B%d" % (layers, B)
+    s.share_layers = layers
+    return s
+
+
 def profile_decode(B=8, L=65536, seed=0x5EED + 5) -> Spec:
     """bf16 decode, batch B at context L: a profiling case larger than L2 (0.75 GB resident)."""
     return Spec("profile_decode_bf16_B%d_L%d" % (B, L), lens=[L] * B, q_req=list(range(B)),
@@ -254,6 +279,8 @@ WORKLOADS = {
     "batched_decode": batched_decode,
     "prefill": prefill,
     "long_decode": long_decode,
+    "short_decode": short_decode,
+    "indexshare": indexshare,
     "profile_decode": profile_decode,
     "profile_prefill": profile_prefill,
     "profile_long": profile_long,
@@ -291,4 +318,6 @@ def subset(inputs: dict, queries: List[int]) -> dict:
             out[name] = inputs[name][dev_ids].cpu()
         elif name in inputs:
             out[name] = None
+    out["shared"] = [{"q_mla": sh["q_mla"][qi.to(sh["q_mla"].device)].cpu(),
+                      "latent_pool": sh["latent_pool"][dev_ids].cpu()} for sh in inputs.get("shared", [])]
     return out

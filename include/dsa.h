@@ -151,8 +151,13 @@ dsa_status dsa_indexer_topk(const void* q, int32_t q_dtype, int32_t Hi, int32_t 
  *   lse[t,h]   = ln sum_j exp(logit_j)          (-inf and out = 0 when nothing is selected)
  * Entries idx[t,j] == -1 are skipped; any other index outside 0..q_pos[t] sets
  * DSA_DEVERR_INDEX and is skipped.
+ * Dense case (same page, section "Lightning Indexer": a query that sees fewer than K positions
+ * keeps all of them): idx == NULL attends every visible position 0..q_pos[t], with no selection;
+ * then k >= max_context is required (k bounds the rows per query).  A caller whose queries all
+ * see at most K positions skips the indexer and the selection and calls this directly.
  * q: device [num_queries, H, d_v + d_rope] of q_dtype; latent: paged cache with
- * dim == d_v + d_rope and dtype == q_dtype (f32 or bf16); idx: device int32 [num_queries, k];
+ * dim == d_v + d_rope and dtype == q_dtype (f32 or bf16); idx: device int32 [num_queries, k]
+ * or NULL (dense);
  * out: device [num_queries, H, d_v] of q_dtype; lse: device f32 [num_queries, H] or NULL.
  * workspace: device scratch of at least dsa_mla_workspace_size(num_queries, H, d_v, k) bytes,
  * 256-byte aligned (may be NULL when that size is 0).

@@ -197,28 +197,31 @@ def dsa_indexer_topk(q, w, keys: PagedCache, batch: Batch, k, scores, idx, strea
     return idx
 
 
-def _mla(fn_name, q, latent: PagedCache, batch: Batch, idx, softmax_scale, out, lse, workspace, stream):
+def _mla(fn_name, q, latent: PagedCache, batch: Batch, idx, softmax_scale, out, lse, workspace, stream, k=None):
     lib = load_library()
     T, H, dqk = q.shape
     d_v = out.shape[-1]
     lc, bc = latent._c(), batch._c()
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    if k is None:
+        k = idx.shape[1] if idx is not None else int(batch.max_context)
     _check(getattr(lib, fn_name)(_dev_ptr(q, "q"), _dtype_code(q), H, d_v, dqk - d_v, ctypes.byref(lc),
-                                 ctypes.byref(bc), _dev_ptr(idx, "idx"), idx.shape[1], float(softmax_scale),
+                                 ctypes.byref(bc), _dev_ptr(idx, "idx"), int(k), float(softmax_scale),
                                  _dev_ptr(out, "out"), _dev_ptr(lse, "lse"), _dev_ptr(workspace, "workspace"),
                                  ws_bytes, _stream(stream)))
     return out
 
 
 def dsa_sparse_mla_decode(q, latent: PagedCache, batch: Batch, idx, softmax_scale, out, lse=None,
-                          workspace=None, stream=None):
-    """Sparse MQA-mode MLA over the selected latent rows, split-K across CTAs (include/dsa.h)."""
-    return _mla("dsa_sparse_mla_decode", q, latent, batch, idx, softmax_scale, out, lse, workspace, stream)
+                          workspace=None, stream=None, k=None):
+    """Sparse MQA-mode MLA over the selected latent rows, split-K across CTAs (include/dsa.h).
+    ``idx=None`` is the dense case: every visible position, with k (default max_context) rows."""
+    return _mla("dsa_sparse_mla_decode", q, latent, batch, idx, softmax_scale, out, lse, workspace, stream, k)
 
 
 def dsa_sparse_mla_prefill(q, latent: PagedCache, batch: Batch, idx, softmax_scale, out, lse=None,
-                           workspace=None, stream=None):
-    return _mla("dsa_sparse_mla_prefill", q, latent, batch, idx, softmax_scale, out, lse, workspace, stream)
+                           workspace=None, stream=None, k=None):
+    return _mla("dsa_sparse_mla_prefill", q, latent, batch, idx, softmax_scale, out, lse, workspace, stream, k)
 
 
 def dsa_sparse_mla_decode_noalloc(q, latent: PagedCache, batch: Batch, idx, softmax_scale, out, lse=None,

@@ -289,7 +289,9 @@ static dsa_status mla_common(bool decode, const void* q, int32_t q_dtype, int32_
   if (st != DSA_OK) return st;
   if (batch->num_queries == 0) return DSA_OK;
   if ((st = check_cache(latent, batch, "latent")) != DSA_OK) return st;
-  if (!q || !idx || !out) return fail(DSA_ERR_INVALID_ARG, "mla: NULL q, idx or out%s");
+  if (!q || !out) return fail(DSA_ERR_INVALID_ARG, "mla: NULL q or out%s");
+  if (!idx && k < batch->max_context)
+    return fail(DSA_ERR_INVALID_ARG, "mla: without a selection (idx NULL) k must be >= max_context%s");
   if (H < 1 || d_v < 1 || d_rope < 0) return fail(DSA_ERR_INVALID_ARG, "mla: bad H, d_v or d_rope%s");
   if (d_v > 1024 || d_v + d_rope > 4096) return fail(DSA_ERR_INVALID_ARG, "mla: d_v <= 1024 and d_v + d_rope <= 4096 required%s");
   if (latent->dim != d_v + d_rope) return fail(DSA_ERR_INVALID_ARG, "mla: latent dim != d_v + d_rope%s");

@@ -103,8 +103,10 @@ __global__ void mla_generic_kernel(MlaArgs a) {
   float o[kMaxVPerThread];
 #pragma unroll
   for (int c = 0; c < kMaxVPerThread; ++c) o[c] = 0.0f;
-  for (int j = 0; j < a.k; ++j) {
-    const int p = a.idx[(int64_t)t * a.k + j];
+  // without a selection (idx null) every visible position is attended: slot j holds position j
+  const int nslots = a.idx ? a.k : min(a.k, pos + 1);
+  for (int j = 0; j < nslots; ++j) {
+    const int p = a.idx ? a.idx[(int64_t)t * a.k + j] : j;
     if (p == -1) continue;
     if (p < -1 || p > pos) {
       if (threadIdx.x == 0 && h == 0) raise_error(a.err, DSA_DEVERR_INDEX);

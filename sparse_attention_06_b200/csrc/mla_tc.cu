@@ -99,6 +99,7 @@ struct Params {
   int64_t num_blocks;
   int32_t oob_row;               // first row past the pool (gathered as zeros)
   int T, k, ks, nsplit, num_reqs, max_blocks, max_context;
+  bool dense;                    // no selection (idx null): every visible position, slot j = position j
   float scale_log2;              // softmax scale * log2(e)
   int* err;
 };
@@ -128,13 +129,14 @@ constexpr int kNoSlot = -2;
 // pos_block applies that gate where the position is used, a tile later.)
 __device__ __forceinline__ int slot_pos(const Params& p, int t, int sp, int slot) {
   if (slot >= min(p.k, (sp + 1) * p.ks)) return kNoSlot;
+  if (p.dense) return slot;
   return p.idx[(int64_t)t * p.k + slot];
 }
 // ... and the physical block holding it (-1 when unused or out of range; flagged when `report`).
 __device__ __forceinline__ int pos_block(const Params& p, bool qok, int req, int pos, int ps, bool report) {
   if (!qok || ps == kNoSlot || ps == -1) return -1;
   if (ps < 0 || ps > pos) {
-    if (report) raise_error(p.err, DSA_DEVERR_INDEX);
+    if (report && !p.dense) raise_error(p.err, DSA_DEVERR_INDEX);  // dense: slots past the query are unused
     return -1;
   }
   const int lblk = ps / kPage;
@@ -159,9 +161,12 @@ __device__ __forceinline__ uint8_t* q_stage_box(uint8_t* smem, int c) {
   return c < 4 ? smem + OFF_K + K_BYTES + c * Q_CHUNK : smem + OFF_P;
 }
 
-__device__ __forceinline__ int unit_tiles(const Params& p, int sp) {
+// 64-row tiles of unit (t, sp): its split's share of the k selection slots, or, without a
+// selection, of the query's visible positions.
+__device__ __forceinline__ int unit_tiles(const Params& p, int t, int sp) {
   const int first = sp * p.ks;
-  const int n = min(p.ks, p.k - first);
+  const int slots = p.dense ? min(p.k, max(0, p.q_pos[t] + 1)) : p.k;
+  const int n = min(p.ks, slots - first);
   return n > 0 ? (n + kTile - 1) / kTile : 0;
 }
 
@@ -327,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int req = p.q_req[t];
       const int pos = p.q_pos[t];
       const bool qok = req >= 0 && req < p.num_reqs && pos >= 0 && pos < p.max_context;
-      const int ntiles = unit_tiles(p, sp);
+      const int ntiles = unit_tiles(p, t, sp);
       const bool mine = lane < kKeysPerWarp;
       const int kslot = sp * p.ks + gw * kKeysPerWarp + lane;
       int ps_j = mine && ntiles > 0 ? slot_pos(p, t, sp, kslot) : kNoSlot;
@@ -429,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
         int t, sp, v;
         unit_coords(p, u, t, sp, v);
-        const int ntiles = unit_tiles(p, sp);
+        const int ntiles = unit_tiles(p, t, sp);
         if constexpr (staged_q) {
           if (!(ok = mbar_wait(q_first, 0, p.err, abort_flag))) break;
         } else {
@@ -487,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         int t, sp, v;
         unit_coords(p, u, t, sp, v);
-        const int ntiles = unit_tiles(p, sp);
+        const int ntiles = unit_tiles(p, t, sp);
         for (int j = 0; j < ntiles; ++j) {
           const int g = gi + j, s = g % kStages;
           if (!(ok = mbar_wait(p_full, g & 1, p.err, abort_flag))) break;
@@ -552,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       int t, sp, v;
       unit_coords(p, u, t, sp, v);
-      const int ntiles = unit_tiles(p, sp);
+      const int ntiles = unit_tiles(p, t, sp);
       float m_used = -INFINITY, l = 0.0f;
       for (int j = 0; j < ntiles; ++j) {
         const int g = gi + j, s = g % kStages;
@@ -787,6 +792,7 @@ cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_
   p.latent = static_cast<const __nv_bfloat16*>(a.latent.data);
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.idx = a.idx;
+  p.dense = a.idx == nullptr;
   p.q_req = a.batch.q_req;
   p.q_pos = a.batch.q_pos;
   p.block_table = a.batch.block_table;

@@ -45,3 +45,13 @@ def test_work_model_prefill_row_gather_hbm_bytes():
     assert m["mla_hbm_rows"] == 65536 + 4096
     dec = bench.work_model(di.batched_decode())
     assert dec["mla_hbm_rows"] == dec["mla_rows"] == 64 * 2048
+
+
+def test_work_model_dense_and_indexshare():
+    short = bench.work_model(di.short_decode())
+    assert short["indexer_bytes"] == 0 and short["topk_bytes"] == 0      # the dense case: no indexer
+    assert short["mla_rows"] == sum(L for L in di.short_decode().lens)   # every visible position
+    one = bench.work_model(di.batched_decode())
+    grp = bench.work_model(di.indexshare())
+    assert grp["indexer_bytes"] == one["indexer_bytes"]                  # one indexer per group
+    assert grp["mla_flops"] == 4 * one["mla_flops"] and grp["mla_bytes"] == 4 * one["mla_bytes"]

@@ -10,7 +10,7 @@ import torch
 import dsa_inputs as di
 import oracle
 import sparse_attention_06_b200 as dsa
-from _parity import TOL, check_topk, parity_case, to_dev
+from _parity import TOL, cache_and_batch, check_mla, check_topk, parity_case, run_gpu, subset_cpu, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -267,3 +267,71 @@ def test_bounded_wait_runs_out_and_context_stays_usable():
     spec = _spec([2300], seed=33)
     x = to_dev(di.generate(spec, "cpu"))
     parity_case(x, kind="bf16")
+
+
+# ---------------------------------------------------------------------------------------------
+# the dense case and IndexShare
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("entry", ["decode", "prefill"])
+def test_dense_case_without_selection(entry):
+    # every query sees at most K positions, so the method keeps them all: sparse MLA with no
+    # selection (idx None) over the visible positions equals the oracle's attention over all of
+    # them, and, bit for bit, the sparse path whose selection is then every position
+    lens = [1500, 2048, 700, 64, 1999, 130]
+    spec = _spec(lens, seed=17)
+    x = to_dev(di.generate(spec, "cpu"))
+    g = run_gpu(x, entry)
+    assert g["err"] == 0
+    keys, lat, batch, max_ctx = cache_and_batch(x)
+    out = torch.full_like(g["out"], float("nan"))
+    lse = torch.full_like(g["lse"], float("nan"))
+    ws_bytes = dsa.dsa_mla_workspace_size(spec.T, spec.H, spec.d_v, spec.k)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda") if ws_bytes else None
+    fn = dsa.dsa_sparse_mla_decode if entry == "decode" else dsa.dsa_sparse_mla_prefill
+    dsa.dsa_clear_device_error()
+    fn(x["q_mla"], lat, batch, None, spec.scale, out, lse, ws, k=spec.k)
+    assert dsa.dsa_get_device_error() == 0
+    assert torch.equal(out, g["out"]) and torch.equal(lse, g["lse"])
+    j = np.arange(spec.k)[None, :]
+    n = np.array(lens)[:, None]
+    idx_all = np.where(j < n, j, -1).astype(np.int32)
+    sub = subset_cpu(x, list(range(spec.T)))
+    ora_out, ora_lse = oracle.sparse_mla(sub["q_mla"], sub["latent_pool"], sub["block_table"], sub["q_req"],
+                                         idx_all, spec.d_v, spec.scale)
+    check_mla(out.float().cpu(), lse.cpu(), ora_out, ora_lse, TOL["bf16"])
+
+
+def test_dense_case_needs_k_covering_the_context():
+    spec = _spec([3000], seed=19)
+    x = to_dev(di.generate(spec, "cpu"))
+    keys, lat, batch, max_ctx = cache_and_batch(x)
+    out = torch.empty((1, spec.H, spec.d_v), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.dsa_sparse_mla_decode(x["q_mla"], lat, batch, None, spec.scale, out, k=2048)
+    assert e.value.status == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_indexshare_layers_reuse_the_selection():
+    # one full layer selects; the group's other layers (own queries and latent caches, same
+    # requests and paging) attend over the cached selection
+    spec = di.Spec("share", lens=[5000, 3000, 2100, 9000], q_req=[0, 1, 2, 3], q_pos=[4999, 2999, 2099, 8999],
+                   share_layers=3, seed=18)
+    x = to_dev(di.generate(spec, "cpu"))
+    g = run_gpu(x)
+    assert g["err"] == 0
+    keys, lat, batch, max_ctx = cache_and_batch(x)
+    ws_bytes = dsa.dsa_mla_workspace_size(spec.T, spec.H, spec.d_v, spec.k)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda") if ws_bytes else None
+    sub = subset_cpu(x, list(range(spec.T)))
+    assert len(x["shared"]) == 2
+    for sh, sh_cpu in zip(x["shared"], sub["shared"]):
+        out = torch.empty_like(g["out"])
+        lse = torch.empty_like(g["lse"])
+        dsa.dsa_clear_device_error()
+        dsa.dsa_sparse_mla_decode(sh["q_mla"], dsa.PagedCache(sh["latent_pool"]), batch, g["idx"].cuda(),
+                                  spec.scale, out, lse, ws)
+        assert dsa.dsa_get_device_error() == 0
+        ora_out, ora_lse = oracle.sparse_mla(sh_cpu["q_mla"], sh_cpu["latent_pool"], sub["block_table"],
+                                             sub["q_req"], g["idx"].cpu(), spec.d_v, spec.scale)
+        check_mla(out.float().cpu(), lse.cpu(), ora_out, ora_lse, TOL["bf16"])
