@@ -3,8 +3,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl dsa|reference]
 
 One step is one pass of the whole hot path over one batch of synthetic, seeded input: indexer
-scores (dsa_indexer_scores), top-K selection (dsa_topk_select) and sparse MLA
-(dsa_sparse_mla_decode, or dsa_sparse_mla_prefill for the prefill chunk).  The default workload
+scores fused with the top-K selection (dsa_indexer_topk with its histogram workspace) and sparse
+MLA (dsa_sparse_mla_decode, or dsa_sparse_mla_prefill for the prefill chunk).  The default workload
 is batched bf16 decode: 64 requests with context lengths uniform in [4096, 131072], paged in
 64-token blocks with shuffled block tables (indexer 64 heads x 128, top-2048, MLA 128 heads over
 512 + 64) -- the largest single-GPU workload by bytes.  Other workloads: tiny, decode (batch 1,
@@ -73,7 +73,8 @@ def work_model(spec):
         r = spec.q_req[t]
         per_req[r] = max(per_req.get(r, 0), vis[t])
     key_tokens = sum(per_req.values())
-    idx_bytes = key_tokens * key_bytes_per_token(spec) + T * spec.Hi * (spec.Di * act + 4) + pairs * 4
+    q_bytes = spec.Di + 4 if spec.q_idx_dtype == "e4m3" else spec.Di * act  # per head (+ its scale)
+    idx_bytes = key_tokens * key_bytes_per_token(spec) + T * spec.Hi * (q_bytes + 4) + pairs * 4
     idx_flops = 2.0 * pairs * spec.Hi * spec.Di
     sel = [min(v, spec.k) for v in vis]
     topk_bytes = pairs * 4 + T * spec.k * 4
@@ -252,6 +253,9 @@ class Layer:
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev) if ws else None
         self.prefill = spec.query_group > 1
         self.q_idx, self.w, self.q_mla = x["q_idx"], x["w"], x["q_mla"]
+        self.q_scale = x.get("q_idx_scale")
+        # the fused selection's histogram workspace: zero-filled once, every call leaves it zeroed
+        self.khist = torch.zeros(dsa.dsa_indexer_topk_workspace_size(spec.T) // 4, dtype=torch.int32, device=dev)
         # every query sees at most K positions: the method keeps them all, so the layer is
         # attention over the whole context without indexer or selection (the dense case)
         self.dense = self.max_ctx <= spec.k
@@ -266,14 +270,30 @@ class Layer:
         fn(q, lat, self.batch, idx, self.spec.scale, out, lse, self.ws, k=self.spec.k)
 
     def step_sparse(self, ev=None):
-        """Indexer -> top-K -> sparse MLA (and the shared layers' sparse MLA on the same selection)."""
+        """Indexer fused with the top-K selection (the indexer builds each query's order-key digit
+        histogram, the selection places its threshold from it and clears it) -> sparse MLA (and
+        the shared layers' sparse MLA on the same selection).  With events (per-kernel breakdown)
+        the two kernels of the fused call are enqueued by their own entry points, same arguments."""
         d = self.dsa
-        d.dsa_indexer_scores(self.q_idx, self.w, self.keys, self.batch, self.scores)
-        if ev is not None:
+        if ev is None:
+            d.dsa_indexer_topk(self.q_idx, self.w, self.keys, self.batch, self.spec.k, self.scores, self.idx,
+                               q_scale=self.q_scale, workspace=self.khist)
+        else:
+            d.dsa_indexer_scores(self.q_idx, self.w, self.keys, self.batch, self.scores, q_scale=self.q_scale,
+                                 key_hist=self.khist)
             ev[0].record()
-        d.dsa_topk_select(self.scores, self.batch.q_pos, self.spec.k, self.idx)
-        if ev is not None:
+            d.dsa_topk_select(self.scores, self.batch.q_pos, self.spec.k, self.idx, key_hist=self.khist)
             ev[1].record()
+        self._mla(self.q_mla, self.lat, self.out, self.lse, self.idx)
+        for q, lat, out, lse in self.shared:
+            self._mla(q, lat, out, lse, self.idx)
+
+    def step_unfused(self):
+        """The same layer with the selection sampling its threshold (no histogram from the
+        indexer): the comparison for the fused indexer-selection path."""
+        d = self.dsa
+        d.dsa_indexer_scores(self.q_idx, self.w, self.keys, self.batch, self.scores, q_scale=self.q_scale)
+        d.dsa_topk_select(self.scores, self.batch.q_pos, self.spec.k, self.idx)
         self._mla(self.q_mla, self.lat, self.out, self.lse, self.idx)
         for q, lat, out, lse in self.shared:
             self._mla(q, lat, out, lse, self.idx)
@@ -288,9 +308,8 @@ class Layer:
 
     def step_full_layer(self):
         """One full layer alone (indexer, top-K, sparse MLA): the IndexShare comparison."""
-        d = self.dsa
-        d.dsa_indexer_scores(self.q_idx, self.w, self.keys, self.batch, self.scores)
-        d.dsa_topk_select(self.scores, self.batch.q_pos, self.spec.k, self.idx)
+        self.dsa.dsa_indexer_topk(self.q_idx, self.w, self.keys, self.batch, self.spec.k, self.scores, self.idx,
+                                  q_scale=self.q_scale, workspace=self.khist)
         self._mla(self.q_mla, self.lat, self.out, self.lse, self.idx)
 
 
@@ -391,6 +410,8 @@ def run_cuda(args):
     # end to end through the public API: per-step query-side inputs from pinned host memory,
     # the KV caches resident in HBM (state), output read back every step
     names = ("q_req", "q_pos", "block_table", "q_mla") + (() if layer.dense else ("q_idx", "w"))
+    if not layer.dense and x.get("q_idx_scale") is not None:
+        names += ("q_idx_scale",)
 
     def query_inputs(c):  # device tensors of one copy that the host supplies every step
         return [c[n] for n in names] + [sh["q_mla"] for sh in c.get("shared", [])]
@@ -421,17 +442,24 @@ def run_cuda(args):
     peaks = load_peaks()
     tensor_peak = peaks["bf16_tflops_sustained"] if statistics.mean(step_ms_sep) > 50 else peaks["bf16_tflops"]
     roofs = {}
-    for name, ms_list, nbytes, flops in (("indexer", idx_ms, model["indexer_bytes"], model["indexer_flops"]),
-                                         ("topk", topk_ms, model["topk_bytes"], 0.0),
-                                         ("mla", mla_ms, model["mla_bytes"], model["mla_flops"])):
+    # e4m3 x e4m3 indexer products run at twice the bf16 rate: their peak is the measured bf16
+    # peak times the nominal fp8 / bf16 ratio (2)
+    idx_peak_mult = 2.0 if spec.q_idx_dtype == "e4m3" else 1.0
+    for name, ms_list, nbytes, flops, pmult in (
+            ("indexer", idx_ms, model["indexer_bytes"], model["indexer_flops"], idx_peak_mult),
+            ("topk", topk_ms, model["topk_bytes"], 0.0, 1.0),
+            ("mla", mla_ms, model["mla_bytes"], model["mla_flops"], 1.0)):
         if nbytes == 0 and flops == 0:
             continue  # not run in this workload (the dense case has no indexer or selection)
         t = statistics.mean(ms_list) / 1e3
         t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
-        t_ten = flops / (tensor_peak * 1e12)
+        t_ten = flops / (pmult * tensor_peak * 1e12)
         if t_ten > t_hbm:
-            roofs[name] = {"bound": "tensor", "achieved": flops / t / 1e12, "peak": tensor_peak,
-                           "unit": "TFLOP/s", "frac": flops / t / 1e12 / tensor_peak, "us": t * 1e6}
+            pk = pmult * tensor_peak
+            roofs[name] = {"bound": "tensor", "achieved": flops / t / 1e12, "peak": pk,
+                           "unit": "TFLOP/s", "frac": flops / t / 1e12 / pk, "us": t * 1e6}
+            if pmult != 1.0:
+                roofs[name]["peak_note"] = "fp8: measured bf16 peak x 2 (nominal fp8/bf16 ratio)"
         else:
             roofs[name] = {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": peaks["hbm_gbs"],
                            "unit": "GB/s", "frac": nbytes / t / 1e9 / peaks["hbm_gbs"], "us": t * 1e6}
@@ -452,6 +480,9 @@ def run_cuda(args):
         sp_ms = _time_steps(lambda i: layers[i % ncopy].step_sparse(), K, stream) / K
         breakdown["sparse_path_us"] = sp_ms * 1e3
         breakdown["dense_saving"] = 1.0 - ms_per_step / sp_ms
+    if not layer.dense:
+        uf_ms = _time_steps(lambda i: layers[i % ncopy].step_unfused(), K, stream) / K
+        breakdown["layer_us_selection_unfused"] = uf_ms * 1e3
     if layer.shared:
         fl_ms = _time_steps(lambda i: layers[i % ncopy].step_full_layer(), K, stream) / K
         n_l = 1 + len(layer.shared)
@@ -510,7 +541,7 @@ def oracle_step(sub, spec, nthreads):
         idx = np.where(j < n[:, None], j, -1).astype(np.int32)
     else:
         s = oracle.indexer_scores(sub["q_idx"], sub["w"], sub["key_pool"], sub["key_scale"], sub["block_table"],
-                                  sub["q_req"], sub["q_pos"], nthreads=nthreads)
+                                  sub["q_req"], sub["q_pos"], nthreads=nthreads, q_scale=sub.get("q_idx_scale"))
         idx = oracle.topk(s, sub["q_pos"], spec.k, nthreads=nthreads)
     oracle.sparse_mla(sub["q_mla"], sub["latent_pool"], sub["block_table"], sub["q_req"], idx, spec.d_v,
                       spec.scale, nthreads=nthreads)
@@ -608,7 +639,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="batched_decode",
                     choices=["tiny", "decode", "batched_decode", "prefill", "long_decode", "short_decode",
-                             "indexshare", "profile_decode", "profile_prefill", "profile_long"])
+                             "indexshare", "prefill_q8", "long_decode_q8", "profile_decode", "profile_prefill",
+                             "profile_long"])
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -8,7 +8,8 @@ Recipe (every tensor has its own generator seeded from (seed, tensor id, chunk))
     N(0, 1) rounded to the stored dtype (bf16 RNE, or f32 for the tiny workload);
   * indexer head weights w [T, Hi] ~ U(0, 1), f32;
   * e4m3 indexer keys: per-token scale = max_i |k_i| / 448 (f32), code = RNE(k / scale) clamped
-    to +-448 -- the quantisation happens here, once; both sides read the same bytes;
+    to +-448 -- the quantisation happens here, once; both sides read the same bytes; e4m3 indexer
+    queries (the fp8-query workloads) are quantised the same way per (query, head);
   * paged pools of 64-token blocks; each request's logical blocks are mapped to a random
     permutation of the physical blocks (shuffled block tables), unused entries are -1;
   * planted heavy tail (long-context workload): a seeded 2% of each request's positions get their
@@ -51,6 +52,7 @@ class Spec:
     seed: int = 0x5EED
     query_group: int = 1       # queries come in runs of this many sharing one request
     share_layers: int = 1      # layers in an IndexShare group: one full layer, the rest reuse its selection
+    q_idx_dtype: str = ""      # "" (act_dtype) or "e4m3": indexer queries quantised per (query, head)
 
     @property
     def T(self) -> int:
@@ -154,7 +156,12 @@ def generate(spec: Spec, device="cpu", with_mla=True, with_indexer=True):
             out["key_pool"] = kraw.to(_dt(spec.key_dtype)).view(nblk, BLOCK, spec.Di)
             out["key_scale"] = None
         del kraw
-        out["q_idx"] = q_idx
+        if spec.q_idx_dtype == "e4m3":
+            codes, qscale = quantize_e4m3(q_idx)
+            out["q_idx"] = codes
+            out["q_idx_scale"] = qscale
+        else:
+            out["q_idx"] = q_idx
         out["w"] = w
     if with_mla:
         out["q_mla"] = normal((spec.T, spec.H, spec.dqk), act, dev, spec.seed, 4)
@@ -256,6 +263,22 @@ def indexshare(B=64, lo=4096, hi=131072, layers=4, seed=0x5EED + 2) -> Spec:
     return s
 
 
+def prefill_q8(ctx=65536, chunk=4096, seed=0x5EED + 3) -> Spec:
+    """The prefill chunk with e4m3 indexer queries (per-(query, head) scale) as well as e4m3 keys."""
+    s = prefill(ctx, chunk, seed)
+    s.name = "prefill_e4m3q_%dq_ctx%d" % (chunk, ctx)
+    s.q_idx_dtype = "e4m3"
+    return s
+
+
+def long_decode_q8(B=16, L=202752, seed=0x5EED + 4) -> Spec:
+    """Long-context decode with e4m3 indexer queries (per-(query, head) scale) and e4m3 keys."""
+    s = long_decode(B, L, seed)
+    s.name = "long_decode_e4m3q_B%d_L%d" % (B, L)
+    s.q_idx_dtype = "e4m3"
+    return s
+
+
 def profile_decode(B=8, L=65536, seed=0x5EED + 5) -> Spec:
     """bf16 decode, batch B at context L: a profiling case larger than L2 (0.75 GB resident)."""
     return Spec("profile_decode_bf16_B%d_L%d" % (B, L), lens=[L] * B, q_req=list(range(B)),
@@ -281,6 +304,8 @@ WORKLOADS = {
     "long_decode": long_decode,
     "short_decode": short_decode,
     "indexshare": indexshare,
+    "prefill_q8": prefill_q8,
+    "long_decode_q8": long_decode_q8,
     "profile_decode": profile_decode,
     "profile_prefill": profile_prefill,
     "profile_long": profile_long,
@@ -309,15 +334,15 @@ def subset(inputs: dict, queries: List[int]) -> dict:
         "q_pos": torch.tensor([spec.q_pos[t] for t in queries], dtype=torch.int32),
     }
     qi = torch.tensor(queries, dtype=torch.long)
-    dev_ids = ids.to(inputs["block_table"].device)
-    for name in ("q_idx", "w", "q_mla"):
+    for name in ("q_idx", "q_idx_scale", "w", "q_mla"):
         if name in inputs and inputs[name] is not None:
             out[name] = inputs[name][qi.to(inputs[name].device)].cpu()
     for name in ("key_pool", "key_scale", "latent_pool"):
         if name in inputs and inputs[name] is not None:
-            out[name] = inputs[name][dev_ids].cpu()
+            out[name] = inputs[name][ids.to(inputs[name].device)].cpu()
         elif name in inputs:
             out[name] = None
     out["shared"] = [{"q_mla": sh["q_mla"][qi.to(sh["q_mla"].device)].cpu(),
-                      "latent_pool": sh["latent_pool"][dev_ids].cpu()} for sh in inputs.get("shared", [])]
+                      "latent_pool": sh["latent_pool"][ids.to(sh["latent_pool"].device)].cpu()}
+                     for sh in inputs.get("shared", [])]
     return out

@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define DSA_ABI_VERSION 1
+#define DSA_ABI_VERSION 2
 
 typedef enum dsa_status {
   DSA_OK = 0,
@@ -107,15 +107,26 @@ typedef struct dsa_batch {
  * no softmax).
  *   scores[t * ld + s] = sum_h w[t,h] * max(0, sum_i q[t,h,i] * khat[s,i]),  0 <= s <= q_pos[t]
  *   khat = key row (f32/bf16), or e4m3 code * per-token scale.
- * q: device [num_queries, Hi, Di] of q_dtype (DSA_F32 or DSA_BF16); w: device [num_queries, Hi]
- * f32; keys: paged indexer-key cache with dim == Di, same block table as the batch;
- * scores: device f32 [num_queries, ld], ld >= max_context.  Entries s > q_pos[t] are not
- * written.  Fast path: Hi == 64, Di == 128, bf16 q, bf16 or e4m3 keys.
+ *   q[t,h,:] as stored (f32/bf16), or e4m3 code * q_scale[t,h].
+ * q: device [num_queries, Hi, Di] of q_dtype (DSA_F32, DSA_BF16 or DSA_E4M3); q_scale: device f32
+ * [num_queries, Hi] for DSA_E4M3 queries (per query and head), ignored otherwise; w: device
+ * [num_queries, Hi] f32; keys: paged indexer-key cache with dim == Di, same block table as the
+ * batch; scores: device f32 [num_queries, ld], ld >= max_context.  Entries s > q_pos[t] are not
+ * written.  Tensor-core path: Hi == 64, Di == 128, and bf16 q with bf16 or e4m3 keys, or e4m3 q
+ * with e4m3 keys; bf16 queries take any bf16 value (with e4m3 keys each head row is carried as
+ * two e4m3 terms at a power-of-two scale, exact to bf16 precision for every element down to 2^-10
+ * of the row's largest).  Other combinations run on the generic kernels.
+ * key_hist: NULL, or device uint32 [num_queries, 4096] (16-byte aligned) to which the call adds,
+ * per query, how many of its scores fall in each bin of the top 12 bits of the selection's
+ * order key (the key dsa_topk_select compares: sign, exponent and three mantissa bits of the
+ * score); dsa_topk_select takes it to place its threshold.  It is filled by the tensor-core
+ * kernel for bf16 keys with query_group 1 and by the generic kernels; the other tensor-core
+ * configurations leave it untouched.
  */
-dsa_status dsa_indexer_scores(const void* q, int32_t q_dtype, int32_t Hi, int32_t Di,
-                              const float* w, const dsa_paged_cache* keys,
+dsa_status dsa_indexer_scores(const void* q, int32_t q_dtype, const float* q_scale, int32_t Hi,
+                              int32_t Di, const float* w, const dsa_paged_cache* keys,
                               const dsa_batch* batch, float* scores, int64_t ld,
-                              dsa_stream stream);
+                              uint32_t* key_hist, dsa_stream stream);
 
 /*
  * Top-K selection (same page, section "Lightning Indexer": the K highest indexer scores are
@@ -128,19 +139,33 @@ dsa_status dsa_indexer_scores(const void* q, int32_t q_dtype, int32_t Hi, int32_
  * scores: device f32 [T, ld]; q_pos: device int32 [T] with q_pos[t] < ld (a larger value sets
  * DSA_DEVERR_REQUEST and only the first ld scores are used); idx: device int32 [T, k].
  * k in [1, 4096].  Needs no scratch memory.
+ * key_hist: NULL, or the order-key digit histogram of each row's scores as dsa_indexer_scores
+ * builds it ([T, 4096] uint32, 16-byte aligned): the call places its threshold from it instead of
+ * sampling the row, and leaves it zero-filled for the next call.  The result never depends on
+ * it: a histogram that does not match the scores only costs time.
  */
 dsa_status dsa_topk_select(const float* scores, int64_t ld, const int32_t* q_pos, int32_t T,
-                           int32_t k, int32_t* idx, dsa_stream stream);
+                           int32_t k, int32_t* idx, uint32_t* key_hist, dsa_stream stream);
 
 /*
- * Indexer scores followed by the top-K selection, in one call.  `scores` is caller-owned
- * scratch of [num_queries, ld] f32 (ld >= max_context) that receives the scores; idx is
- * device int32 [num_queries, k].  Same arguments and semantics as the two calls above.
+ * Indexer scores fused with the top-K selection (same page, section "Lightning Indexer": the
+ * indexer exists to pick each query's top K).  `scores` is caller-owned scratch of
+ * [num_queries, ld] f32 (ld >= max_context) that receives the scores; idx is device int32
+ * [num_queries, k].  Same semantics as the two calls above.  With a workspace of
+ * dsa_indexer_topk_workspace_size(num_queries) bytes (16-byte aligned) the indexer kernel builds
+ * each query's order-key digit histogram as it writes the scores (where dsa_indexer_scores
+ * fills key_hist), and the selection takes its threshold from it (no sampling pass); the
+ * workspace must be zero-filled before its first use and every call leaves it zero-filled
+ * again.  Without a workspace, or where the indexer builds no histogram, the selection samples.
  */
-dsa_status dsa_indexer_topk(const void* q, int32_t q_dtype, int32_t Hi, int32_t Di,
-                            const float* w, const dsa_paged_cache* keys,
+dsa_status dsa_indexer_topk(const void* q, int32_t q_dtype, const float* q_scale, int32_t Hi,
+                            int32_t Di, const float* w, const dsa_paged_cache* keys,
                             const dsa_batch* batch, int32_t k, float* scores, int64_t ld,
-                            int32_t* idx, dsa_stream stream);
+                            int32_t* idx, void* workspace, size_t workspace_bytes,
+                            dsa_stream stream);
+
+/* Bytes of the dsa_indexer_topk workspace for num_queries queries (4096 uint32 counters each). */
+size_t dsa_indexer_topk_workspace_size(int32_t num_queries);
 
 /*
  * Sparse MLA in MQA mode over the selected rows (same page, sections "Sparse MLA" and "MLA

@@ -49,7 +49,7 @@ def _load():
         if _lib is None:
             lib = ctypes.CDLL(build())
             P, I, L, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
-            lib.oracle_indexer_scores.argtypes = [I, P, I, I, I, P, P, I, P, I, P, I, P, P, P, L, I]
+            lib.oracle_indexer_scores.argtypes = [I, P, I, P, I, I, P, P, I, P, I, P, I, P, P, P, L, I]
             lib.oracle_topk.argtypes = [I, P, L, P, I, P, I]
             lib.oracle_sparse_mla.argtypes = [I, P, I, I, I, I, P, I, I, P, I, P, P, I, D, P, P, I]
             lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
@@ -99,13 +99,14 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
 
-def indexer_scores(q, w, key_pool, key_scale, block_table, q_req, q_pos, ld=None, nthreads=0):
+def indexer_scores(q, w, key_pool, key_scale, block_table, q_req, q_pos, ld=None, nthreads=0, q_scale=None):
     """Lightning-indexer scores in fp64 (page "How GLM5.3 Sparse Attention Affects HBM Memory
     Usage", section "Lightning Indexer").
 
-    q [T, Hi, Di] (f32/bf16), w [T, Hi] f32, key_pool [num_blocks, block_size, Di] (f32/bf16/e4m3),
-    key_scale [num_blocks, block_size] f32 or None, block_table [B, max_blocks] i32,
-    q_req [T] i32, q_pos [T] i32.  Returns float64 [T, ld]; entries past q_pos[t] are NaN.
+    q [T, Hi, Di] (f32/bf16, or e4m3 codes with q_scale [T, Hi] f32), w [T, Hi] f32,
+    key_pool [num_blocks, block_size, Di] (f32/bf16/e4m3), key_scale [num_blocks, block_size] f32
+    or None, block_table [B, max_blocks] i32, q_req [T] i32, q_pos [T] i32.  Returns float64
+    [T, ld]; entries past q_pos[t] are NaN.
     """
     qa, qdt = _raw(q)
     wa, _ = _raw(w)
@@ -113,6 +114,11 @@ def indexer_scores(q, w, key_pool, key_scale, block_table, q_req, q_pos, ld=None
     T, Hi, Di = qa.shape
     nblk, bs, Dk = ka.shape
     assert Dk == Di and wa.shape == (T, Hi) and wa.dtype == np.float32
+    if qdt == E4M3:
+        qsa = np.ascontiguousarray(_raw(q_scale)[0], dtype=np.float32)
+        assert qsa.shape == (T, Hi)
+    else:
+        qsa = np.zeros(1, np.float32)
     if kdt == E4M3:
         sa, _ = _raw(key_scale)
         sa = np.ascontiguousarray(sa, dtype=np.float32)
@@ -126,7 +132,7 @@ def indexer_scores(q, w, key_pool, key_scale, block_table, q_req, q_pos, ld=None
         ld = int(qp.max()) + 1 if T else 1
     out = np.full((T, ld), np.nan, dtype=np.float64)
     _load().oracle_indexer_scores(
-        T, _ptr(qa), qdt, Hi, Di, _ptr(wa), _ptr(ka), kdt, _ptr(sa), bs, _ptr(bt), bt.shape[1],
+        T, _ptr(qa), qdt, _ptr(qsa), Hi, Di, _ptr(wa), _ptr(ka), kdt, _ptr(sa), bs, _ptr(bt), bt.shape[1],
         _ptr(qr), _ptr(qp), _ptr(out), ld, nthreads,
     )
     return out

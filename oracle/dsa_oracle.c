@@ -20,7 +20,8 @@
  * Readings taken where the pages are silent (each is also listed in the design notes):
  *   - visibility is causal including the query's own position: query t sees 0..q_pos[t];
  *   - no constant scaling inside the indexer (a caller folds any constant into w);
- *   - e4m3 keys are dequantised as e4m3_value * per-token scale before the dot product;
+ *   - e4m3 keys are dequantised as e4m3_value * per-token scale before the dot product, and e4m3
+ *     queries as e4m3_value * per-(query, head) scale;
  *   - ties in the top-K are broken by the lower position; -0.0 equals +0.0;
  *   - selected positions are emitted in ascending order, padded with -1 when fewer than K;
  *   - LSE is the natural-log log-sum-exp of the scaled logits.
@@ -99,20 +100,25 @@ int oracle_max_threads(void) {
 
 /*
  * Lightning indexer scores.
- *   out[t, s] = sum_h w[t,h] * max(0, sum_i q[t,h,i] * khat[s,i])      for 0 <= s <= q_pos[t]
+ *   out[t, s] = sum_h w[t,h] * max(0, sum_i qhat[t,h,i] * khat[s,i])   for 0 <= s <= q_pos[t]
  *   khat[s,i] = key[row(s), i] * (key dtype is e4m3 ? key_scale[row(s)] : 1)
+ *   qhat[t,h,i] = q[t,h,i] * (q dtype is e4m3 ? q_scale[t,h] : 1)
  * Entries s > q_pos[t] are left untouched.
- * q: [T, Hi, Di] of q_dtype; w: [T, Hi] f32; key pool: [num_blocks * block_size, Di] of k_dtype;
- * key_scale: [num_blocks * block_size] f32 (e4m3 only).
+ * q: [T, Hi, Di] of q_dtype; q_scale: [T, Hi] f32 (e4m3 queries only); w: [T, Hi] f32;
+ * key pool: [num_blocks * block_size, Di] of k_dtype; key_scale: [num_blocks * block_size] f32
+ * (e4m3 only).
  */
-void oracle_indexer_scores(int T, const void* q, int q_dtype, int Hi, int Di, const float* w,
+void oracle_indexer_scores(int T, const void* q, int q_dtype, const float* q_scale, int Hi, int Di, const float* w,
                            const void* kpool, int k_dtype, const float* key_scale, int block_size,
                            const int32_t* block_table, int max_blocks, const int32_t* q_req,
                            const int32_t* q_pos, double* out, int64_t ld, int nthreads) {
   set_threads(nthreads);
   double* qt = (double*)malloc(sizeof(double) * (size_t)Hi * (size_t)Di);
   for (int t = 0; t < T; ++t) {
-    for (int64_t e = 0; e < (int64_t)Hi * Di; ++e) qt[e] = load_elem(q, q_dtype, (int64_t)t * Hi * Di + e);
+    for (int64_t e = 0; e < (int64_t)Hi * Di; ++e) {
+      double qs = (q_dtype == OR_E4M3) ? (double)q_scale[(int64_t)t * Hi + e / Di] : 1.0;
+      qt[e] = load_elem(q, q_dtype, (int64_t)t * Hi * Di + e) * qs;
+    }
     int64_t n = (int64_t)q_pos[t] + 1;
     /* the key positions of one query are independent: they are shared out among the threads */
 #pragma omp parallel

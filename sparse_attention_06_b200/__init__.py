@@ -35,6 +35,7 @@ EXPORTED = (
     "dsa_sparse_mla_prefill", "dsa_mla_workspace_size", "dsa_get_device_error",
     "dsa_clear_device_error", "dsa_status_string", "dsa_last_error_message", "dsa_abi_version",
     "dsa_kernel_launch_count", "dsa_sparse_mla_decode_noalloc", "dsa_selftest_bounded_wait",
+    "dsa_indexer_topk_workspace_size",
 )
 
 
@@ -77,9 +78,9 @@ def load_library():
     P, I32, I64, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
     PC, PB = ctypes.POINTER(_PagedCache), ctypes.POINTER(_Batch)
     sig = {
-        "dsa_indexer_scores": [P, I32, I32, I32, P, PC, PB, P, I64, P],
-        "dsa_topk_select": [P, I64, P, I32, I32, P, P],
-        "dsa_indexer_topk": [P, I32, I32, I32, P, PC, PB, I32, P, I64, P, P],
+        "dsa_indexer_scores": [P, I32, P, I32, I32, P, PC, PB, P, I64, P, P],
+        "dsa_topk_select": [P, I64, P, I32, I32, P, P, P],
+        "dsa_indexer_topk": [P, I32, P, I32, I32, P, PC, PB, I32, P, I64, P, P, ctypes.c_size_t, P],
         "dsa_sparse_mla_decode": [P, I32, I32, I32, I32, PC, PB, P, I32, F, P, P, P, ctypes.c_size_t, P],
         "dsa_sparse_mla_prefill": [P, I32, I32, I32, I32, PC, PB, P, I32, F, P, P, P, ctypes.c_size_t, P],
         "dsa_sparse_mla_decode_noalloc": [P, I32, I32, I32, I32, PC, PB, P, I32, F, P, P, P],
@@ -93,6 +94,8 @@ def load_library():
         fn.restype = ctypes.c_int
     lib.dsa_mla_workspace_size.argtypes = [I32, I32, I32, I32]
     lib.dsa_mla_workspace_size.restype = ctypes.c_size_t
+    lib.dsa_indexer_topk_workspace_size.argtypes = [I32]
+    lib.dsa_indexer_topk_workspace_size.restype = ctypes.c_size_t
     lib.dsa_status_string.argtypes = [ctypes.c_int]
     lib.dsa_status_string.restype = ctypes.c_char_p
     lib.dsa_last_error_message.restype = ctypes.c_char_p
@@ -168,33 +171,46 @@ class Batch:
                       int(self.query_group), 0)
 
 
-def dsa_indexer_scores(q, w, keys: PagedCache, batch: Batch, scores, stream=None):
-    """scores[t, s] = sum_h w[t,h] ReLU(q[t,h] . khat[s]) for s <= q_pos[t] (include/dsa.h)."""
+def dsa_indexer_scores(q, w, keys: PagedCache, batch: Batch, scores, stream=None, q_scale=None, key_hist=None):
+    """scores[t, s] = sum_h w[t,h] ReLU(qhat[t,h] . khat[s]) for s <= q_pos[t] (include/dsa.h);
+    e4m3 queries (uint8 codes) come with q_scale [T, Hi] f32; key_hist [T, 4096] int32/uint32
+    (optional) receives the scores' order-key digit counts."""
     lib = load_library()
     T, Hi, Di = q.shape
     kc, bc = keys._c(), batch._c()
-    _check(lib.dsa_indexer_scores(_dev_ptr(q, "q"), _dtype_code(q), Hi, Di, _dev_ptr(w, "w"),
-                                  ctypes.byref(kc), ctypes.byref(bc), _dev_ptr(scores, "scores"),
-                                  scores.shape[1], _stream(stream)))
+    _check(lib.dsa_indexer_scores(_dev_ptr(q, "q"), _dtype_code(q), _dev_ptr(q_scale, "q_scale"), Hi, Di,
+                                  _dev_ptr(w, "w"), ctypes.byref(kc), ctypes.byref(bc), _dev_ptr(scores, "scores"),
+                                  scores.shape[1], _dev_ptr(key_hist, "key_hist"), _stream(stream)))
     return scores
 
 
-def dsa_topk_select(scores, q_pos, k, idx, stream=None):
-    """idx[t] = the k best positions of scores[t, :q_pos[t]+1], ascending, -1 padded."""
+def dsa_topk_select(scores, q_pos, k, idx, stream=None, key_hist=None):
+    """idx[t] = the k best positions of scores[t, :q_pos[t]+1], ascending, -1 padded; key_hist
+    (optional) places the threshold and is left zeroed (include/dsa.h)."""
     lib = load_library()
     _check(lib.dsa_topk_select(_dev_ptr(scores, "scores"), scores.shape[1], _dev_ptr(q_pos, "q_pos"),
-                               q_pos.numel(), k, _dev_ptr(idx, "idx"), _stream(stream)))
+                               q_pos.numel(), k, _dev_ptr(idx, "idx"), _dev_ptr(key_hist, "key_hist"),
+                               _stream(stream)))
     return idx
 
 
-def dsa_indexer_topk(q, w, keys: PagedCache, batch: Batch, k, scores, idx, stream=None):
+def dsa_indexer_topk(q, w, keys: PagedCache, batch: Batch, k, scores, idx, stream=None, q_scale=None,
+                     workspace=None):
+    """Indexer scores fused with the top-K selection; workspace (optional, zero-filled before its
+    first use, left zero-filled) holds the order-key digit histograms (include/dsa.h)."""
     lib = load_library()
     T, Hi, Di = q.shape
     kc, bc = keys._c(), batch._c()
-    _check(lib.dsa_indexer_topk(_dev_ptr(q, "q"), _dtype_code(q), Hi, Di, _dev_ptr(w, "w"),
-                                ctypes.byref(kc), ctypes.byref(bc), k, _dev_ptr(scores, "scores"),
-                                scores.shape[1], _dev_ptr(idx, "idx"), _stream(stream)))
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib.dsa_indexer_topk(_dev_ptr(q, "q"), _dtype_code(q), _dev_ptr(q_scale, "q_scale"), Hi, Di,
+                                _dev_ptr(w, "w"), ctypes.byref(kc), ctypes.byref(bc), k, _dev_ptr(scores, "scores"),
+                                scores.shape[1], _dev_ptr(idx, "idx"), _dev_ptr(workspace, "workspace"), ws_bytes,
+                                _stream(stream)))
     return idx
+
+
+def dsa_indexer_topk_workspace_size(num_queries) -> int:
+    return int(load_library().dsa_indexer_topk_workspace_size(num_queries))
 
 
 def _mla(fn_name, q, latent: PagedCache, batch: Batch, idx, softmax_scale, out, lse, workspace, stream, k=None):

@@ -43,6 +43,28 @@ __device__ __forceinline__ float load_elem(const void* base, int dtype, int64_t 
 }
 
 // ---------------------------------------------------------------------------------------------
+// order keys of scores (selection) and their digit histogram
+// ---------------------------------------------------------------------------------------------
+// Order-preserving 32-bit key of a score: a larger score has a larger key, -0.0 has the key of
+// +0.0, and NaN gets the lowest key (0) with `is_nan` set.
+__device__ __forceinline__ uint32_t order_key(float f, bool& is_nan) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) {
+    is_nan = true;
+    return 0u;
+  }
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Histogram of order keys by their top kKeyDigitBits bits (sign, exponent and three mantissa
+// bits: eight bins per binade), one row of kKeyBins counters per query.  The indexer adds its
+// scores to it; the selection reads a row to place its threshold and clears it again.
+constexpr int kKeyDigitBits = 12;
+constexpr int kKeyBins = 1 << kKeyDigitBits;
+__device__ __forceinline__ uint32_t key_digit(uint32_t key) { return key >> (32 - kKeyDigitBits); }
+
+// ---------------------------------------------------------------------------------------------
 // shared-memory addresses, mbarriers
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

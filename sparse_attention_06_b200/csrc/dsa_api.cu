@@ -223,10 +223,14 @@ dsa_status dsa_clear_device_error(dsa_stream stream) {
                      "dsa_clear_device_error");
 }
 
-dsa_status dsa_indexer_scores(const void* q, int32_t q_dtype, int32_t Hi, int32_t Di,
-                              const float* w, const dsa_paged_cache* keys,
-                              const dsa_batch* batch, float* scores, int64_t ld,
-                              dsa_stream stream) {
+// The indexer call behind dsa_indexer_scores; *hist_built tells whether the launched kernel adds
+// the scores to key_hist (the generic kernel and the tensor-core kernel for one query per tile
+// with bf16 keys do; the others leave it untouched).
+static dsa_status indexer_scores_impl(const void* q, int32_t q_dtype, const float* q_scale, int32_t Hi,
+                                      int32_t Di, const float* w, const dsa_paged_cache* keys,
+                                      const dsa_batch* batch, float* scores, int64_t ld,
+                                      uint32_t* key_hist, dsa_stream stream, bool* hist_built) {
+  *hist_built = false;
   dsa_status st = check_batch(batch);
   if (st != DSA_OK) return st;
   if (batch->num_queries == 0) return DSA_OK;
@@ -234,50 +238,83 @@ dsa_status dsa_indexer_scores(const void* q, int32_t q_dtype, int32_t Hi, int32_
   if (!q || !w || !scores) return fail(DSA_ERR_INVALID_ARG, "indexer: NULL q, w or scores%s");
   if (Hi < 1 || Di < 1 || Hi * Di > 16384) return fail(DSA_ERR_INVALID_ARG, "indexer: Hi*Di must be in [1, 16384]%s");
   if (keys->dim != Di) return fail(DSA_ERR_INVALID_ARG, "indexer: key dim != Di%s");
-  if (q_dtype != DSA_F32 && q_dtype != DSA_BF16) return fail(DSA_ERR_INVALID_ARG, "indexer: q dtype must be f32 or bf16%s");
+  if (q_dtype != DSA_F32 && q_dtype != DSA_BF16 && q_dtype != DSA_E4M3)
+    return fail(DSA_ERR_INVALID_ARG, "indexer: q dtype must be f32, bf16 or e4m3%s");
+  if (q_dtype == DSA_E4M3 && !q_scale) return fail(DSA_ERR_INVALID_ARG, "indexer: e4m3 q needs q_scale%s");
   if (ld < batch->max_context) return fail(DSA_ERR_INVALID_ARG, "indexer: ld < max_context%s");
+  if (key_hist && !aligned16(key_hist)) return fail(DSA_ERR_INVALID_ARG, "indexer: key_hist not 16-byte aligned%s");
   int* err;
   int sms;
   if (!device_state(&err, &sms)) return fail(DSA_ERR_CUDA, "no CUDA device%s");
-  IndexerArgs a{q, q_dtype, Hi, Di, w, *keys, *batch, scores, ld, err};
-  const bool tc_shape = Hi == 64 && Di == 128 && q_dtype == DSA_BF16 && keys->block_size == 64 &&
-                        (keys->dtype == DSA_BF16 || keys->dtype == DSA_E4M3) && aligned16(q) &&
+  IndexerArgs a{q, q_dtype, q_dtype == DSA_E4M3 ? q_scale : nullptr, Hi, Di, w, *keys, *batch, scores, ld,
+                key_hist, err};
+  // tensor-core operand pairs: bf16 x bf16, e4m3 keys x bf16 queries, e4m3 x e4m3
+  const bool tc_pair = (q_dtype == DSA_BF16 && (keys->dtype == DSA_BF16 || keys->dtype == DSA_E4M3)) ||
+                       (q_dtype == DSA_E4M3 && keys->dtype == DSA_E4M3);
+  const bool tc_shape = Hi == 64 && Di == 128 && tc_pair && keys->block_size == 64 && aligned16(q) &&
                         (ld % 4) == 0 && aligned16(scores);
   cudaError_t e;
-  if (tc_shape && batch->query_group % 4 == 0)
+  if (tc_shape && batch->query_group % 4 == 0) {
     e = launch_indexer_tc_prefill(a, sms, static_cast<cudaStream_t>(stream));
-  else if (tc_shape)
+  } else if (tc_shape) {
     e = launch_indexer_tc_decode(a, sms, static_cast<cudaStream_t>(stream));
-  else
+    *hist_built = key_hist && keys->dtype == DSA_BF16;
+  } else {
     e = launch_indexer_generic(a, static_cast<cudaStream_t>(stream));
+    *hist_built = key_hist != nullptr;
+  }
   return cuda_status(e, "dsa_indexer_scores launch", 1);
 }
 
+dsa_status dsa_indexer_scores(const void* q, int32_t q_dtype, const float* q_scale, int32_t Hi,
+                              int32_t Di, const float* w, const dsa_paged_cache* keys,
+                              const dsa_batch* batch, float* scores, int64_t ld,
+                              uint32_t* key_hist, dsa_stream stream) {
+  bool built;
+  return indexer_scores_impl(q, q_dtype, q_scale, Hi, Di, w, keys, batch, scores, ld, key_hist, stream, &built);
+}
+
 dsa_status dsa_topk_select(const float* scores, int64_t ld, const int32_t* q_pos, int32_t T,
-                           int32_t k, int32_t* idx, dsa_stream stream) {
+                           int32_t k, int32_t* idx, uint32_t* key_hist, dsa_stream stream) {
   if (T < 0) return fail(DSA_ERR_INVALID_ARG, "topk: T < 0%s");
   if (T == 0) return DSA_OK;
   if (!scores || !q_pos || !idx) return fail(DSA_ERR_INVALID_ARG, "topk: NULL pointer%s");
   if (k < 1 || k > 4096) return fail(DSA_ERR_INVALID_ARG, "topk: k must be in [1, 4096]%s");
   if (ld < 1) return fail(DSA_ERR_INVALID_ARG, "topk: ld < 1%s");
+  if (key_hist && !aligned16(key_hist)) return fail(DSA_ERR_INVALID_ARG, "topk: key_hist not 16-byte aligned%s");
   int* err;
   int sms;
   if (!device_state(&err, &sms)) return fail(DSA_ERR_CUDA, "no CUDA device%s");
-  return cuda_status(launch_topk(scores, ld, q_pos, T, k, idx, err, static_cast<cudaStream_t>(stream)),
+  return cuda_status(launch_topk(scores, ld, q_pos, T, k, idx, key_hist, err, static_cast<cudaStream_t>(stream)),
                      "dsa_topk_select launch", 1);
 }
 
-dsa_status dsa_indexer_topk(const void* q, int32_t q_dtype, int32_t Hi, int32_t Di,
-                            const float* w, const dsa_paged_cache* keys,
+dsa_status dsa_indexer_topk(const void* q, int32_t q_dtype, const float* q_scale, int32_t Hi,
+                            int32_t Di, const float* w, const dsa_paged_cache* keys,
                             const dsa_batch* batch, int32_t k, float* scores, int64_t ld,
-                            int32_t* idx, dsa_stream stream) {
+                            int32_t* idx, void* workspace, size_t workspace_bytes,
+                            dsa_stream stream) {
   dsa_status st = check_batch(batch);
   if (st != DSA_OK) return st;
   if (batch->num_queries == 0) return DSA_OK;
   if (!idx) return fail(DSA_ERR_INVALID_ARG, "indexer_topk: idx is NULL%s");
   if (k < 1 || k > 4096) return fail(DSA_ERR_INVALID_ARG, "indexer_topk: k must be in [1, 4096]%s");
-  if ((st = dsa_indexer_scores(q, q_dtype, Hi, Di, w, keys, batch, scores, ld, stream)) != DSA_OK) return st;
-  return dsa_topk_select(scores, ld, batch->q_pos, batch->num_queries, k, idx, stream);
+  uint32_t* key_hist = nullptr;
+  if (workspace) {
+    if (workspace_bytes < dsa_indexer_topk_workspace_size(batch->num_queries) || !aligned16(workspace))
+      return fail(DSA_ERR_INVALID_ARG, "indexer_topk: workspace too small or not 16-byte aligned%s");
+    key_hist = static_cast<uint32_t*>(workspace);
+  }
+  bool built = false;
+  if ((st = indexer_scores_impl(q, q_dtype, q_scale, Hi, Di, w, keys, batch, scores, ld, key_hist, stream,
+                                &built)) != DSA_OK)
+    return st;
+  // the selection takes the histogram only when the indexer kernel built it (else it samples)
+  return dsa_topk_select(scores, ld, batch->q_pos, batch->num_queries, k, idx, built ? key_hist : nullptr, stream);
+}
+
+size_t dsa_indexer_topk_workspace_size(int32_t num_queries) {
+  return num_queries > 0 ? (size_t)num_queries * kKeyBins * sizeof(uint32_t) : 0;
 }
 
 static dsa_status mla_common(bool decode, const void* q, int32_t q_dtype, int32_t H, int32_t d_v,

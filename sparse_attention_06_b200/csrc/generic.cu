@@ -4,7 +4,8 @@
 // indexer 4 heads x 32, MLA 8 heads over 64 + 16) and serve as the bring-up path.  They follow
 // the definitions directly:
 //   indexer (page "How GLM5.3 Sparse Attention Affects HBM Memory Usage", section "Lightning
-//   Indexer"): score = sum_h w_h * ReLU(q_h . khat), khat = key * per-token scale for e4m3;
+//   Indexer"): score = sum_h w_h * ReLU(q_h . khat), khat = key * per-token scale for e4m3
+//   (e4m3 queries likewise: qhat = code * per-(query, head) scale);
 //   sparse MLA (same page, "Sparse MLA"): softmax over the selected rows of scale * q . row,
 //   output = softmax-weighted sum of the rows' first d_v dims, computed with a running max.
 #include <math.h>
@@ -48,8 +49,10 @@ __global__ void indexer_generic_kernel(IndexerArgs a) {
   }
   const int64_t s0 = (int64_t)blockIdx.x * kGenericTile;
   if (s0 > pos) return;  // uniform over the block
-  for (int e = threadIdx.x; e < a.Hi * a.Di; e += blockDim.x)
-    qs[e] = load_elem(a.q, a.q_dtype, (int64_t)t * a.Hi * a.Di + e);
+  for (int e = threadIdx.x; e < a.Hi * a.Di; e += blockDim.x) {
+    const float qsc = a.q_scale ? a.q_scale[(int64_t)t * a.Hi + e / a.Di] : 1.0f;  // e4m3 queries
+    qs[e] = load_elem(a.q, a.q_dtype, (int64_t)t * a.Hi * a.Di + e) * qsc;
+  }
   for (int h = threadIdx.x; h < a.Hi; h += blockDim.x) ws[h] = a.w[(int64_t)t * a.Hi + h];
   __syncthreads();
   const int64_t s = s0 + threadIdx.x;
@@ -67,6 +70,10 @@ __global__ void indexer_generic_kernel(IndexerArgs a) {
     score = fmaf(ws[h], fmaxf(dot, 0.0f), score);
   }
   a.scores[(int64_t)t * a.ld + s] = score;
+  if (a.key_hist) {  // the selection's threshold histogram
+    bool nan = false;
+    atomicAdd(&a.key_hist[(int64_t)t * kKeyBins + key_digit(order_key(score, nan))], 1u);
+  }
 }
 
 constexpr int kMlaThreads = 128;

@@ -14,12 +14,14 @@ namespace dsa {
 struct IndexerArgs {
   const void* q;
   int q_dtype;
+  const float* q_scale;  // [T, Hi] for e4m3 queries, else null
   int Hi, Di;
   const float* w;
   dsa_paged_cache keys;
   dsa_batch batch;
   float* scores;
   int64_t ld;
+  uint32_t* key_hist;  // [T, kKeyBins] order-key digit counts to add to, or null
   int* err;
 };
 
@@ -43,9 +45,10 @@ struct MlaArgs {
 cudaError_t launch_indexer_generic(const IndexerArgs& a, cudaStream_t s);
 cudaError_t launch_mla_generic(const MlaArgs& a, cudaStream_t s);
 
-// radix top-k (any k <= 4096)
+// radix top-k (any k <= 4096); key_hist (or null): [T, kKeyBins] digit counts of each row's
+// scores, read to place the threshold and left zeroed
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, int T, int k,
-                        int32_t* idx, int* err, cudaStream_t s);
+                        int32_t* idx, uint32_t* key_hist, int* err, cudaStream_t s);
 
 // tcgen05 paths (production shapes)
 cudaError_t launch_indexer_tc_decode(const IndexerArgs& a, int num_sms, cudaStream_t s);

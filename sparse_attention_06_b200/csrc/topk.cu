@@ -10,16 +10,23 @@
 // C CTAs (C = 1..8, chosen so that rows x C fills the SMs); CTA r owns a contiguous slice of the
 // row's positions.
 //
-//   1. Threshold.  Every CTA reads the same strided sample of the row (8-score chunks; the loads
-//      of its own slice are already in flight) and finds, by radix steps of 12-bit digits, a key
-//      tau with at least js sample keys >= tau, js = rk + 4 sqrt(rk) + 8 where rk is the sample
-//      rank of the row's K-th score: the count of sample keys above that score is about binomial
-//      with mean rk, so fewer than K candidates (and the exact path below) needs a deviation of
-//      more than four standard deviations (~1e-6 per row).  Rows of at most kCap positions take
-//      every score (no threshold).
-//   2. Filter.  One coalesced pass over the slice appends every (key, position) with
-//      score >= tau to shared memory (one shared atomic per warp and 256 scores), and the CTA
-//      stores its candidate count into every CTA of the cluster.
+//   1. Threshold.  With the row's order-key digit histogram (12-bit digits: the sign, exponent
+//      and three mantissa bits of the score; the indexer builds it as it writes the scores) every
+//      CTA finds the digit bin that holds the row's K-th key, and tau is that bin's lower edge: the
+//      keys >= tau are exactly the keys of that bin and above, whose number the histogram gives.
+//      Without a histogram, or when that number exceeds the candidate capacity, every CTA reads
+//      the same strided sample of the row (8-score chunks) and finds, by radix steps of 12-bit
+//      digits, a key tau with at least js sample keys >= tau, js = rk + 4 sqrt(rk) + 8 where rk
+//      is the sample rank of the row's K-th score: the count of sample keys above that score is
+//      about binomial with mean rk, so fewer than K candidates (and the exact path below) needs a
+//      deviation of more than four standard deviations (~1e-6 per row).  Rows of at most kCap
+//      positions take every score (no threshold).  A histogram that does not describe the row
+//      (one left dirty) only leads to a wrong tau, which step 2's count catches (exact path).
+//      Each CTA clears its share of the histogram row once every CTA has used it.
+//   2. Filter.  One coalesced pass over the slice, two batches of 4096 scores in flight ahead of
+//      the one it filters, appends every (key, position) with score >= tau to shared memory (one
+//      shared atomic per warp and 256 scores), and the CTA stores its candidate count into every
+//      CTA of the cluster.
 //   3. Exact K-th key.  After a cluster barrier every CTA gathers all candidate keys of the row
 //      through distributed shared memory and radix-selects the K-th largest key Tk among them.
 //      If the row had at least K candidates, every score >= Tk is a candidate, so Tk is the
@@ -53,9 +60,13 @@ constexpr int kCap = 6144;                 // candidates of one row (all CTAs of
 constexpr int kMaxSlice = 1 << 17;         // positions one CTA's bitmap covers
 constexpr int kMaxCluster = 8;
 constexpr int kSample = 4096;              // sampled keys (512 chunks of 8)
-constexpr int kPer = 16;                   // scores per thread per filter step
+constexpr int kPer = 16;                   // scores per thread per step of the exact path
+constexpr int kFPer = 8;                   // scores per thread per filter batch
+constexpr int kFStep = kFPer * kThreads;   // scores per filter batch
 static_assert(kHBins == 8 * kThreads, "each thread scans 8 histogram bins");
 static_assert(kCap >= kSample, "the sample fits the key pool");
+static_assert(kKeyBins == 8 * kThreads, "each thread reads 8 bins of a digit histogram row");
+static_assert(kKeyBins % (4 * kMaxCluster) == 0, "every CTA clears whole 16-byte pieces of a histogram row");
 
 struct Smem {
   uint32_t bitmap[kMaxSlice / 32];      // selected positions of this CTA's slice
@@ -115,15 +126,6 @@ __device__ __forceinline__ uint32_t cluster_addr(const void* local, uint32_t ran
   return remote;
 }
 
-// 32-bit load from the shared memory of CTA `rank` of this cluster, at the offset of `local`.
-// Ordered after the last cluster barrier by that barrier's acquire; no compiler barrier here, so
-// that several of these loads can be in flight at once.
-__device__ __forceinline__ uint32_t ld_cluster_u32(const uint32_t* local, uint32_t rank) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr(local, rank)));
-  return v;
-}
-
 // Four consecutive 32-bit words (16-byte aligned) from the shared memory of CTA `rank`.
 __device__ __forceinline__ uint4 ld_cluster_u32x4(const uint32_t* local, uint32_t rank) {
   uint4 v;
@@ -141,16 +143,6 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t* local, uint32_t rank, u
 // ---------------------------------------------------------------------------------------------
 // keys, scans, radix selection
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t order_key(float f, bool& is_nan) {
-  uint32_t u = __float_as_uint(f);
-  if ((u & 0x7FFFFFFFu) > 0x7F800000u) {
-    is_nan = true;
-    return 0u;
-  }
-  if (u == 0x80000000u) u = 0u;
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
 // Inverse of order_key on the keys it produces: the float whose key is `key` (keys below the key
 // of -inf map to a NaN pattern, which no comparison accepts).
 __device__ __forceinline__ float key_to_float(uint32_t key) {
@@ -363,19 +355,19 @@ __device__ __noinline__ void topk_exact(const float* row, int64_t n, int k, int3
 }
 
 // v[j] for a j known only at run time, without indexing the register array
-__device__ __forceinline__ float pick(const float (&v)[kPer], int j) {
+__device__ __forceinline__ float pick(const float (&v)[kFPer], int j) {
   float x = v[0];
 #pragma unroll
-  for (int e = 1; e < kPer; ++e) x = j == e ? v[e] : x;
+  for (int e = 1; e < kFPer; ++e) x = j == e ? v[e] : x;
   return x;
 }
 
-// kPer scores of a slice for this thread, from 16-byte loads where the slice allows: element
+// kFPer scores of a slice for this thread, from 16-byte loads where the slice allows: element
 // j sits at base + ((j / 4) * kThreads + tid) * 4 + j % 4.
-__device__ __forceinline__ void load_batch(const float* srow, int len, int base, bool vec, float (&v)[kPer]) {
+__device__ __forceinline__ void load_batch(const float* srow, int len, int base, bool vec, float (&v)[kFPer]) {
   const int tid = threadIdx.x;
 #pragma unroll
-  for (int u = 0; u < kPer / 4; ++u) {
+  for (int u = 0; u < kFPer / 4; ++u) {
     const int i = base + (u * kThreads + tid) * 4;
     if (vec && i + 4 <= len) {
       const float4 f = __ldg(reinterpret_cast<const float4*>(srow + i));
@@ -387,9 +379,49 @@ __device__ __forceinline__ void load_batch(const float* srow, int len, int base,
   }
 }
 
+// Place of the k-th largest key of a row in its order-key digit histogram (global memory, one
+// row of kKeyBins counters): the bin b holding it, the keys in higher bins and the keys in b.
+// Thread tid owns the 8 bins [8 (kThreads - 1 - tid), 8 (kThreads - tid)), so counts run
+// downward from the top bin (thread 0) to bin 0 (the last thread).  found = false when the
+// histogram holds fewer than k keys.
+struct HistPlace {
+  uint32_t bin, above, count;
+  bool found;
+};
+__device__ __noinline__ HistPlace place_in_histogram(const uint32_t* __restrict__ hrow, uint32_t k) {
+  Smem& S = smem();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint4* mine = reinterpret_cast<const uint4*>(hrow) + 2 * (kThreads - 1 - tid);
+  const uint4 lo4 = __ldg(mine), hi4 = __ldg(mine + 1);
+  const uint32_t h[8] = {hi4.w, hi4.z, hi4.y, hi4.x, lo4.w, lo4.z, lo4.y, lo4.x};
+  const uint32_t lsum = (lo4.x + lo4.y) + (lo4.z + lo4.w) + (hi4.x + hi4.y) + (hi4.z + hi4.w);
+  const uint32_t lincl = warp_inclusive_scan(lsum);
+  if (lane == 31) S.wsum[warp] = lincl;
+  if (tid == 0) S.res[0][3] = 0u;  // found
+  __syncthreads();
+  uint32_t abv = __reduce_add_sync(0xFFFFFFFFu, lane < warp ? S.wsum[lane] : 0u) + lincl - lsum;
+  if (abv < k && k <= abv + lsum) {
+    const int top = kKeyBins - 1 - 8 * tid;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      if (abv < k && k <= abv + h[b]) {
+        S.res[0][0] = (uint32_t)(top - b);
+        S.res[0][1] = abv;
+        S.res[0][2] = h[b];
+        S.res[0][3] = 1u;
+      }
+      abv += h[b];
+    }
+  }
+  __syncthreads();
+  HistPlace r{S.res[0][0], S.res[0][1], S.res[0][2], S.res[0][3] != 0u};
+  __syncthreads();  // res is reused by the radix selections
+  return r;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     topk_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ q_pos, int k,
-                int32_t* __restrict__ idx, int* err) {
+                int32_t* __restrict__ idx, uint32_t* __restrict__ key_hist, int* err) {
   Smem& S = smem();
   const int tid = threadIdx.x, lane = tid & 31;
   griddep_launch_dependents();
@@ -398,20 +430,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   // warm the address translation of this row (a prefetch reads nothing that the previous kernel
   // may still write: the loads below come after the wait)
   if (tid == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(scores + t * ld + min((int64_t)r * 4096, ld - 1)));
-  griddep_wait();  // the scores come from the previous kernel of the stream
+  griddep_wait();  // the scores (and their histogram) come from the previous kernel of the stream
   int64_t n = (int64_t)q_pos[t] + 1;
   if (n > ld) {  // a row cannot hold more scores than its stride
     if (tid == 0 && r == 0) raise_error(err, DSA_DEVERR_REQUEST);
     n = ld;
   }
   int32_t* out = idx + t * k;
+  // The row's digit histogram (when given): read for the threshold below, then this CTA clears its
+  // share of it, once no CTA of the cluster reads it any more, so that it starts at zero next call.
+  uint32_t* hrow = key_hist ? key_hist + t * kKeyBins : nullptr;
+  auto clear_histogram_share = [&]() {
+    if (!hrow) return;
+    const int per = kKeyBins / (int)C;
+    uint4* h4 = reinterpret_cast<uint4*>(hrow + (int)r * per);
+    for (int e = tid; e < per / 4; e += kThreads) h4[e] = make_uint4(0u, 0u, 0u, 0u);
+  };
   if (n <= k) {  // dense: every visible position, then -1 padding
     for (int64_t j = (int64_t)r * kThreads + tid; j < k; j += (int64_t)C * kThreads) out[j] = j < n ? (int32_t)j : -1;
+    clear_histogram_share();
     return;
   }
   const float* row = scores + t * ld;
   if (tid == 0) S.scal[4] = 0u;  // NaN seen
   if (n > (int64_t)kMaxSlice * C) {  // slices too long for the bitmap: exact path on one CTA
+    clear_histogram_share();
     if (r == 0) {
       __syncthreads();  // the NaN flag is clear
       topk_exact(row, n, k, out);
@@ -428,9 +471,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int words = (len + 31) >> 5;
   const float* srow = row + lo;
   const bool vec = ((reinterpret_cast<uintptr_t>(srow) & 15u) == 0);
-  constexpr int kStep = kPer * kThreads;
-  float v[kPer];
-  load_batch(srow, len, 0, vec, v);  // the first batch of this slice, in flight during step 1
+  // the filter below keeps two batches of loads in flight ahead of the one it processes; the
+  // first two are issued now, so that they land during step 1
+  float v0[kFPer], v1[kFPer], v2[kFPer];
+  load_batch(srow, len, 0, vec, v0);
+  load_batch(srow, len, kFStep, vec, v1);
   for (int w = tid; w < words; w += kThreads) S.bitmap[w] = 0u;
   clear_hist(0);
   clear_hist(1);
@@ -441,42 +486,50 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   bool saw_nan = false;
 
-  // 1. threshold from a strided sample (identical in every CTA of the cluster)
+  // 1. threshold (identical in every CTA of the cluster): the lower edge of the digit bin that holds
+  //    the row's K-th key, from the row's histogram when it has one that places at most kCap
+  //    candidates; else from a strided sample
   const bool take_all = n <= kCap;
   float tau_f = -INFINITY;
   if (!take_all) {
-    constexpr int kChunks = kSample / 8;
-    constexpr int kSPT = kSample / kThreads;
-    float sv[kSPT];
-#pragma unroll
-    for (int e = 0; e < kSPT; ++e) {
-      const int s = tid + e * kThreads;
-      const int64_t p = (((int64_t)(s >> 3) * n / kChunks) & ~int64_t(7)) + (s & 7);
-      sv[e] = row[p];
+    bool placed = false;
+    if (hrow) {
+      const HistPlace hp = place_in_histogram(hrow, (uint32_t)k);
+      if (hp.found && hp.above + hp.count <= (uint32_t)kCap) {
+        placed = true;
+        tau_f = key_to_float(hp.bin << (32 - kKeyDigitBits));
+      }
     }
-    // the first batch is consumed here (NaN check), so that its loads complete with the sample's
-    // rather than after step 1
+    if (!placed) {
+      constexpr int kChunks = kSample / 8;
+      constexpr int kSPT = kSample / kThreads;
+      float sv[kSPT];
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) saw_nan |= v[j] != v[j];
+      for (int e = 0; e < kSPT; ++e) {
+        const int s = tid + e * kThreads;
+        const int64_t p = (((int64_t)(s >> 3) * n / kChunks) & ~int64_t(7)) + (s & 7);
+        sv[e] = row[p];
+      }
 #pragma unroll
-    for (int e = 0; e < kSPT; ++e) S.pool[tid + e * kThreads] = order_key(sv[e], saw_nan);
-    __syncthreads();  // sample keys and cleared histograms visible
-    const float rk = (float)k * (float)kSample / (float)n;  // sample rank of the row's K-th score
-    int js = (int)ceilf(rk + 4.f * sqrtf(rk) + 8.f);
-    js = min(js, kSample);
-    tau_f = key_to_float(kth_key(SmemKeys{kSample, false}, (uint32_t)js, false, (uint32_t)(js / 8 + 2)).key);
+      for (int e = 0; e < kSPT; ++e) S.pool[tid + e * kThreads] = order_key(sv[e], saw_nan);
+      __syncthreads();  // sample keys and cleared histograms visible
+      const float rk = (float)k * (float)kSample / (float)n;  // sample rank of the row's K-th score
+      int js = (int)ceilf(rk + 4.f * sqrtf(rk) + 8.f);
+      js = min(js, kSample);
+      tau_f = key_to_float(kth_key(SmemKeys{kSample, false}, (uint32_t)js, false, (uint32_t)(js / 8 + 2)).key);
+    }
   } else {
     __syncthreads();  // the counters are clear
   }
 
-  // 2. filter: append (key, position) of every score >= tau in this slice; the next batch's loads
-  //    are issued before the current batch is processed
-  for (int base = 0; base < len; base += kStep) {
-    float vn[kPer];
-    if (base + kStep < len) load_batch(srow, len, base + kStep, vec, vn);
+  // 2. filter: append (key, position) of every score >= tau in this slice.  The three batch
+  //    registers take turns (no copies between them, which would wait for the loads in flight):
+  //    while one batch is filtered the next two are on their way.
+  auto filter_batch = [&](int base, float (&v)[kFPer], float (&ahead)[kFPer]) {
+    if (base + 2 * kFStep < len) load_batch(srow, len, base + 2 * kFStep, vec, ahead);
     uint32_t mask = 0u;
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) {
+    for (int j = 0; j < kFPer; ++j) {
       const int i = base + ((j >> 2) * kThreads + tid) * 4 + (j & 3);
       const bool valid = i < len;
       saw_nan |= valid && (v[j] != v[j]);
@@ -497,13 +550,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         S.cand_pos[at] = (uint32_t)(lo + base + ((j >> 2) * kThreads + tid) * 4 + (j & 3));
       }
     }
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) v[j] = vn[j];
+  };
+  for (int base = 0; base < len; base += 3 * kFStep) {
+    filter_batch(base, v0, v2);
+    if (base + kFStep < len) filter_batch(base + kFStep, v1, v0);
+    if (base + 2 * kFStep < len) filter_batch(base + 2 * kFStep, v2, v1);
   }
   if (saw_nan) S.scal[4] = 1u;  // benign race: every writer stores 1
   __syncthreads();
   if (tid < (int)C) st_cluster_u32(&S.cnt_all[r], (uint32_t)tid, S.scal[5]);
   cluster_sync();  // A: every CTA's candidates and counts are visible to the cluster
+  clear_histogram_share();  // every CTA of the cluster has placed its threshold
 
   uint32_t m = 0u;  // the row's candidates
   for (int q = 0; q < (int)C; ++q) m += S.cnt_all[q];
@@ -622,7 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, int T, int k,
-                        int32_t* idx, int* err, cudaStream_t s) {
+                        int32_t* idx, uint32_t* key_hist, int* err, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   int dev = 0, sms = 148;
   cudaError_t e = cudaGetDevice(&dev);
@@ -639,7 +696,7 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_pos, i
   cudaLaunchAttribute attrs[2];
   const cudaLaunchConfig_t cfg = launch_config(dim3((unsigned)((int64_t)T * C)), dim3(kThreads), (size_t)smem, s,
                                                attrs, (unsigned)C);
-  return cudaLaunchKernelEx(&cfg, topk_kernel, scores, ld, q_pos, k, idx, err);
+  return cudaLaunchKernelEx(&cfg, topk_kernel, scores, ld, q_pos, k, idx, key_hist, err);
 }
 
 }  // namespace dsa

@@ -26,7 +26,16 @@ TOL = {
 
 
 def to_dev(x, dev="cuda"):
-    return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    """The inputs dict with every tensor (also inside the IndexShare layers' list) on `dev`."""
+    def mv(v):
+        if isinstance(v, torch.Tensor):
+            return v.to(dev)
+        if isinstance(v, list):
+            return [mv(e) for e in v]
+        if isinstance(v, dict):
+            return {k: mv(e) for k, e in v.items()}
+        return v
+    return {k: (mv(v) if k != "spec" else v) for k, v in x.items()}
 
 
 def cache_and_batch(x):
@@ -38,8 +47,11 @@ def cache_and_batch(x):
     return keys, lat, batch, max_ctx
 
 
-def run_gpu(x, mla_entry="decode"):
-    """Run indexer -> top-K -> sparse MLA through the C ABI on cuda tensors.  Returns CPU copies."""
+def run_gpu(x, mla_entry="decode", fused=True):
+    """Run indexer -> top-K -> sparse MLA through the C ABI on cuda tensors (by default the fused
+    indexer-selection call with its histogram workspace, as the benchmark runs it; fused=False runs
+    the two calls without a histogram).  Returns the device results; the histogram workspace must
+    be all zeros again afterwards."""
     spec = x["spec"]
     keys, lat, batch, max_ctx = cache_and_batch(x)
     T = spec.T
@@ -47,8 +59,15 @@ def run_gpu(x, mla_entry="decode"):
     scores = torch.full((T, ld), float("nan"), dtype=torch.float32, device="cuda")
     idx = torch.empty((T, spec.k), dtype=torch.int32, device="cuda")
     dsa.dsa_clear_device_error()
-    dsa.dsa_indexer_scores(x["q_idx"], x["w"], keys, batch, scores)
-    dsa.dsa_topk_select(scores, x["q_pos"], spec.k, idx)
+    if fused:
+        hist = torch.zeros(dsa.dsa_indexer_topk_workspace_size(T) // 4, dtype=torch.int32, device="cuda")
+        dsa.dsa_indexer_topk(x["q_idx"], x["w"], keys, batch, spec.k, scores, idx, q_scale=x.get("q_idx_scale"),
+                             workspace=hist)
+        torch.cuda.synchronize()
+        assert int(hist.abs().sum()) == 0, "the selection left its histogram workspace dirty"
+    else:
+        dsa.dsa_indexer_scores(x["q_idx"], x["w"], keys, batch, scores, q_scale=x.get("q_idx_scale"))
+        dsa.dsa_topk_select(scores, x["q_pos"], spec.k, idx)
     out = torch.empty((T, spec.H, spec.d_v), dtype=x["q_mla"].dtype, device="cuda")
     lse = torch.empty((T, spec.H), dtype=torch.float32, device="cuda")
     ws_bytes = dsa.dsa_mla_workspace_size(T, spec.H, spec.d_v, spec.k)
@@ -60,14 +79,15 @@ def run_gpu(x, mla_entry="decode"):
     return dict(scores=scores, idx=idx, out=out, lse=lse, err=err)
 
 
-def parity_case(x, queries=None, kind="bf16", mla_entry="decode", e2e_min_overlap=0.999, topk_all_rows=False):
+def parity_case(x, queries=None, kind="bf16", mla_entry="decode", e2e_min_overlap=0.999, topk_all_rows=False,
+                fused=True):
     """Full parity of one workload ``x`` (tensors on cuda): GPU path vs the oracle on the queries
     listed (all by default).  With ``topk_all_rows`` the selection of every query (not only the
     listed ones) is checked bit-exactly against the oracle's selection from the GPU's own scores.
     Returns a dict of the measured errors."""
     spec = x["spec"]
     tol = TOL[kind]
-    g = run_gpu(x, mla_entry)
+    g = run_gpu(x, mla_entry, fused)
     assert g["err"] == 0, "device error word %d" % g["err"]
     if topk_all_rows:
         qpos_all = x["q_pos"].cpu().numpy()
@@ -79,7 +99,8 @@ def parity_case(x, queries=None, kind="bf16", mla_entry="decode", e2e_min_overla
     qpos = sub["q_pos"].numpy()
     ld = g["scores"].shape[1]
     ora_scores = oracle.indexer_scores(sub["q_idx"], sub["w"], sub["key_pool"], sub["key_scale"],
-                                       sub["block_table"], sub["q_req"], sub["q_pos"], ld=ld)
+                                       sub["block_table"], sub["q_req"], sub["q_pos"], ld=ld,
+                                       q_scale=sub.get("q_idx_scale"))
     qi = torch.tensor(qs, dtype=torch.long, device="cuda")
     gs = g["scores"][qi].cpu()
     gidx = g["idx"][qi].cpu()
@@ -140,3 +161,20 @@ def check_mla(gpu_out, gpu_lse, ora_out, ora_lse, tol):
         lse_err = float(np.abs(gpu_lse.double().numpy() - ora_lse).max())
         assert lse_err <= tol["lse_abs"], "lse err %.3g" % lse_err
     return max_abs, rel_l2
+
+
+def key_digit_hist(scores, q_pos):
+    """Order-key digit histogram of each row's visible scores, as the indexer builds it for the
+    selection (top 12 bits of the order key: larger score -> larger key, -0 as +0, NaN -> 0):
+    int32 [T, 4096].  Only a hint for the selection's threshold; results never depend on it."""
+    u = scores.contiguous().view(torch.int32).cpu().numpy().view(np.uint32)
+    neg = (u & 0x80000000) != 0
+    key = np.where(neg, ~u, u | 0x80000000).astype(np.uint32)
+    key[u == 0x80000000] = 0x80000000
+    nan = (u & 0x7FFFFFFF) > 0x7F800000
+    key[nan] = 0
+    out = np.zeros((u.shape[0], 4096), dtype=np.int32)
+    for t in range(u.shape[0]):
+        n = int(q_pos[t]) + 1
+        out[t] = np.bincount(key[t, :n] >> 20, minlength=4096)
+    return torch.from_numpy(out)

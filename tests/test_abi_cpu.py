@@ -33,29 +33,37 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.dsa_abi_version() == 1
+    assert lib.dsa_abi_version() == 2
     assert lib.dsa_status_string(dsa.DSA_ERR_INVALID_ARG) == b"invalid argument"
 
 
 def test_invalid_arguments_rejected_on_host(lib):
     # NULL batch
-    st = lib.dsa_indexer_scores(None, 1, 64, 128, None, None, None, None, 0, None)
+    st = lib.dsa_indexer_scores(None, 1, None, 64, 128, None, None, None, None, 0, None, None)
     assert st == dsa.DSA_ERR_INVALID_ARG
     assert b"batch" in lib.dsa_last_error_message()
     # k out of range / NULL pointers in the selection
-    assert lib.dsa_topk_select(None, 10, None, 1, 5, None, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_topk_select(None, 10, None, 1, 5, None, None, None) == dsa.DSA_ERR_INVALID_ARG
     fake = ctypes.c_void_p(16)
-    assert lib.dsa_topk_select(fake, 10, fake, 1, 0, fake, None) == dsa.DSA_ERR_INVALID_ARG
-    assert lib.dsa_topk_select(fake, 10, fake, 1, 5000, fake, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_topk_select(fake, 10, fake, 1, 0, fake, None, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_topk_select(fake, 10, fake, 1, 5000, fake, None, None) == dsa.DSA_ERR_INVALID_ARG
+    # a histogram must be 16-byte aligned
+    assert lib.dsa_topk_select(fake, 10, fake, 1, 5, fake, ctypes.c_void_p(20), None) == dsa.DSA_ERR_INVALID_ARG
     # query_group must divide num_queries
     b = dsa._Batch(6, 1, 16, 16, 16, 4, 256, 4, 0)
     kc = dsa._PagedCache(16, None, 4, 64, 128, dsa.DSA_BF16, 0)
-    st = lib.dsa_indexer_scores(fake, 1, 64, 128, fake, ctypes.byref(kc), ctypes.byref(b), fake, 256, None)
+    st = lib.dsa_indexer_scores(fake, 1, None, 64, 128, fake, ctypes.byref(kc), ctypes.byref(b), fake, 256, None, None)
     assert st == dsa.DSA_ERR_INVALID_ARG and b"query_group" in lib.dsa_last_error_message()
+    # e4m3 queries without their per-head scale
+    b1 = dsa._Batch(1, 1, 16, 16, 16, 4, 256, 1, 0)
+    kc1 = dsa._PagedCache(16, 16, 4, 64, 128, dsa.DSA_E4M3, 0)
+    st = lib.dsa_indexer_scores(fake, dsa.DSA_E4M3, None, 64, 128, fake, ctypes.byref(kc1), ctypes.byref(b1), fake,
+                                256, None, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG and b"q_scale" in lib.dsa_last_error_message()
     # e4m3 cache without a scale
     b = dsa._Batch(1, 1, 16, 16, 16, 4, 256, 1, 0)
     kc = dsa._PagedCache(16, None, 4, 64, 128, dsa.DSA_E4M3, 0)
-    st = lib.dsa_indexer_scores(fake, 1, 64, 128, fake, ctypes.byref(kc), ctypes.byref(b), fake, 256, None)
+    st = lib.dsa_indexer_scores(fake, 1, None, 64, 128, fake, ctypes.byref(kc), ctypes.byref(b), fake, 256, None, None)
     assert st == dsa.DSA_ERR_INVALID_ARG and b"scale" in lib.dsa_last_error_message()
     # latent dim must be d_v + d_rope; scale must be positive
     lc = dsa._PagedCache(16, None, 4, 64, 500, dsa.DSA_BF16, 0)
@@ -75,8 +83,8 @@ def test_invalid_arguments_rejected_on_host(lib):
 
 def test_empty_batch_is_a_noop(lib):
     b = dsa._Batch(0, 0, None, None, None, 0, 0, 1, 0)
-    assert lib.dsa_indexer_scores(None, 1, 64, 128, None, None, ctypes.byref(b), None, 0, None) == dsa.DSA_OK
-    assert lib.dsa_topk_select(None, 1, None, 0, 16, None, None) == dsa.DSA_OK
+    assert lib.dsa_indexer_scores(None, 1, None, 64, 128, None, None, ctypes.byref(b), None, 0, None, None) == dsa.DSA_OK
+    assert lib.dsa_topk_select(None, 1, None, 0, 16, None, None, None) == dsa.DSA_OK
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
@@ -102,3 +110,10 @@ def test_mla_split_plan_and_workspace(lib):
     assert lib.dsa_mla_workspace_size(2, 128, 512, 100) == 0   # two tiles per query: no split
     assert lib.dsa_mla_workspace_size(0, 128, 512, 2048) == 0
     assert lib.dsa_mla_workspace_size(4, 64, 512, 2048) == 0    # not the tensor-core shape
+
+
+def test_indexer_topk_workspace_size(lib):
+    # one row of 4096 uint32 order-key digit counters per query
+    assert lib.dsa_indexer_topk_workspace_size(1) == 4096 * 4
+    assert lib.dsa_indexer_topk_workspace_size(64) == 64 * 4096 * 4
+    assert lib.dsa_indexer_topk_workspace_size(0) == 0

@@ -10,7 +10,7 @@ import torch
 import dsa_inputs as di
 import oracle
 import sparse_attention_06_b200 as dsa
-from _parity import TOL, cache_and_batch, check_mla, check_topk, parity_case, run_gpu, subset_cpu, to_dev
+from _parity import TOL, cache_and_batch, check_mla, check_topk, key_digit_hist, parity_case, run_gpu, subset_cpu, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -59,6 +59,38 @@ def test_decode_small_k_many_tiles():
     parity_case(x, kind="bf16")
 
 
+@pytest.mark.parametrize("entry,group", [("decode", 1), ("prefill", 4)])
+def test_e4m3_queries_with_e4m3_keys(entry, group):
+    # fp8 indexer queries with a per-(query, head) scale and fp8 keys: one e4m3 x e4m3 product per
+    # key tile; one query per tile (decode) and four queries of one request per tile (prefill)
+    if group == 1:
+        spec = _spec([300, 2049, 4133, 9000, 130], key_dtype="e4m3", q_idx_dtype="e4m3", seed=51)
+    else:
+        ctx, chunk = 2990, 64
+        spec = di.Spec("pq8", lens=[ctx + chunk], q_req=[0] * chunk, q_pos=[ctx + t for t in range(chunk)],
+                       key_dtype="e4m3", q_idx_dtype="e4m3", query_group=4, seed=53)
+    x = to_dev(di.generate(spec, "cpu"))
+    assert x["q_idx"].dtype == torch.uint8 and x["q_idx_scale"].shape == (spec.T, 64)
+    parity_case(x, kind="e4m3", mla_entry=entry)
+
+
+@pytest.mark.parametrize("key_dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("magnitude", ["huge_and_tiny_heads", "all_tiny"])
+def test_indexer_queries_of_any_bf16_magnitude(key_dtype, magnitude):
+    # bf16 indexer queries far outside the f16 range: heads scaled up to 1e30 and down to 1e-30
+    # (whose products overflow or vanish in f16), then every head around 2^-100; the e4m3-key path
+    # carries each head at its own power-of-two scale, the bf16 path multiplies as stored
+    spec = _spec([3000, 700, 2100], key_dtype=key_dtype, seed=52)
+    x = di.generate(spec, "cpu")
+    if magnitude == "huge_and_tiny_heads":
+        mult = torch.tensor([1e30, 1e-30, 3e5, 1e-6, 1.0, 7e12, 2.0 ** -20, 1e20] * 8)
+    else:
+        mult = 2.0 ** (-100.0 + torch.arange(64).float() % 8)
+    x["q_idx"] = (x["q_idx"].float() * mult[None, :, None]).to(torch.bfloat16)
+    assert torch.isfinite(x["q_idx"].float()).all()
+    parity_case(to_dev(x), kind=key_dtype)
+
+
 @pytest.mark.parametrize("entry", ["decode", "prefill"])
 def test_prefill_chunk_e4m3(entry):
     ctx, chunk = 1990, 96  # queries straddle the dense/sparse boundary at K = 2048
@@ -81,13 +113,29 @@ def test_prefill_chunk_bf16_two_requests():
 # standalone selection
 # ---------------------------------------------------------------------------------------------
 
-def _topk_gpu(scores, qpos, k):
+HIST_MODE = "none"  # set by test_topk_edge_cases_with_histograms
+
+
+def _topk_gpu(scores, qpos, k, hist_mode=None):
+    """The selection on the GPU.  hist_mode: "none" (threshold from a sample), "exact" (the rows'
+    order-key digit histogram, as the indexer builds it), "garbage" (a histogram that does not
+    match the scores): the result must be the same in every mode, and any histogram given must
+    be zero afterwards."""
+    mode = hist_mode or HIST_MODE
     s = scores.cuda()
     qp = torch.tensor(qpos, dtype=torch.int32, device="cuda")
     idx = torch.empty((len(qpos), k), dtype=torch.int32, device="cuda")
+    hist = None
+    if mode == "exact":
+        hist = key_digit_hist(scores, qpos).cuda()
+    elif mode == "garbage":
+        g = torch.Generator().manual_seed(len(qpos) * 7919 + k)
+        hist = torch.randint(0, 50, (len(qpos), 4096), generator=g, dtype=torch.int32).cuda()
     dsa.dsa_clear_device_error()
-    dsa.dsa_topk_select(s, qp, k, idx)
+    dsa.dsa_topk_select(s, qp, k, idx, key_hist=hist)
     err = dsa.dsa_get_device_error()
+    if hist is not None:
+        assert int(hist.abs().sum()) == 0, "histogram left dirty"
     return idx.cpu(), err
 
 
@@ -335,3 +383,47 @@ def test_indexshare_layers_reuse_the_selection():
         ora_out, ora_lse = oracle.sparse_mla(sh_cpu["q_mla"], sh_cpu["latent_pool"], sub["block_table"],
                                              sub["q_req"], g["idx"].cpu(), spec.d_v, spec.scale)
         check_mla(out.float().cpu(), lse.cpu(), ora_out, ora_lse, TOL["bf16"])
+
+
+@pytest.mark.parametrize("mode", ["exact", "garbage"])
+def test_topk_edge_cases_with_histograms(mode):
+    # every standalone selection case above again, with the threshold placed from a digit
+    # histogram: the exact one the indexer builds, and one that does not describe the scores
+    global HIST_MODE
+    HIST_MODE = mode
+    try:
+        test_topk_planted_tail_long_rows()
+        test_topk_ties_and_signed_zeros()
+        test_topk_dense_boundary_and_padding()
+        test_topk_cluster_shapes()
+        test_topk_ties_straddle_slices()
+        test_topk_skewed_and_equal_long_rows()
+        test_topk_small_tie_groups_in_last_bin()
+        test_topk_threshold_from_a_misleading_sample()
+        test_topk_nan_in_long_row()
+        test_topk_nan_sets_error_word()
+    finally:
+        HIST_MODE = "none"
+
+
+def test_fused_indexer_topk_matches_unfused_and_reuses_workspace():
+    # the fused call (histogram built by the indexer) against the two plain calls, twice in a row
+    # on the same workspace; bf16 and e4m3 keys, several requests with ragged lengths
+    for key_dtype, seed in (("bf16", 61), ("e4m3", 62)):
+        spec = _spec([40000, 2049, 9000, 130000, 300], key_dtype=key_dtype, seed=seed)
+        x = to_dev(di.generate(spec, "cpu"))
+        keys, lat, batch, max_ctx = cache_and_batch(x)
+        ld = (max_ctx + 3) // 4 * 4
+        scores = torch.empty((spec.T, ld), dtype=torch.float32, device="cuda")
+        ref = torch.empty((spec.T, spec.k), dtype=torch.int32, device="cuda")
+        dsa.dsa_clear_device_error()
+        dsa.dsa_indexer_topk(x["q_idx"], x["w"], keys, batch, spec.k, scores, ref)
+        ws = torch.zeros(dsa.dsa_indexer_topk_workspace_size(spec.T) // 4, dtype=torch.int32, device="cuda")
+        for _ in range(2):
+            idx = torch.full_like(ref, -7)
+            dsa.dsa_indexer_topk(x["q_idx"], x["w"], keys, batch, spec.k, scores, idx, workspace=ws)
+            torch.cuda.synchronize()
+            assert torch.equal(idx, ref)
+            assert int(ws.abs().sum()) == 0
+        assert dsa.dsa_get_device_error() == 0
+        check_topk(ref.cpu(), scores.cpu(), [L - 1 for L in spec.lens], spec.k)

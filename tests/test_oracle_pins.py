@@ -298,3 +298,22 @@ def test_mla_rope_dims_enter_logits_but_not_values():
     np.testing.assert_allclose(a, b, rtol=1e-12)
     c, _ = oracle.sparse_mla(x["q_mla"], x["latent_pool"], x["block_table"], x["q_req"], idx, spec.d_v, spec.scale)
     assert np.abs(c - a).max() > 1e-3
+
+
+def test_indexer_e4m3_queries_dequantise_per_head():
+    # e4m3 query codes with a per-(query, head) scale are the queries code * scale: with
+    # power-of-two scales (exact in f32) the scores equal those of the f32 queries holding the same
+    # values, and a head-index slip in the scale (distinct per head) would break the equality;
+    # scores are degree-1 homogeneous in a common positive query scale
+    x = di.generate(di.tiny(), "cpu")
+    codes, _ = di.quantize_e4m3(x["q_idx"])
+    T, Hi, Di = codes.shape
+    scale = (2.0 ** torch.tensor([[-3.0, 0.0, 2.0, 5.0]])).expand(T, Hi).contiguous().float()
+    qf = (codes.view(torch.float8_e4m3fn).float() * scale.unsqueeze(-1)).contiguous()
+    args = (x["key_pool"], None, x["block_table"], x["q_req"], x["q_pos"])
+    s_q8 = oracle.indexer_scores(codes, x["w"], *args, q_scale=scale)
+    s_f = oracle.indexer_scores(qf, x["w"], *args)
+    assert np.array_equal(s_q8, s_f)
+    s_3 = oracle.indexer_scores(codes, x["w"], *args, q_scale=scale * 3.0)
+    n = int(x["q_pos"][0]) + 1
+    assert np.allclose(s_3[0, :n], 3.0 * s_q8[0, :n], rtol=1e-12, atol=0)
