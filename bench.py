@@ -639,8 +639,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="batched_decode",
                     choices=["tiny", "decode", "batched_decode", "prefill", "long_decode", "short_decode",
-                             "indexshare", "prefill_q8", "long_decode_q8", "profile_decode", "profile_prefill",
-                             "profile_long"])
+                             "indexshare", "prefill_q8", "long_decode_q8", "glm5_decode", "profile_decode",
+                             "profile_prefill", "profile_long"])
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -279,6 +279,17 @@ def long_decode_q8(B=16, L=202752, seed=0x5EED + 4) -> Spec:
     return s
 
 
+def glm5_decode(B=64, lo=4096, hi=131072, seed=0x5EED + 9) -> Spec:
+    """Batched decode with the GLM-5 attention shape: 64 MLA heads over the same 512 + 64 latent
+    rows, softmax scale 1/sqrt(256) (its head dimension); indexer and selection as in the batched
+    decode workload."""
+    s = batched_decode(B, lo, hi, seed)
+    s.name = "glm5_decode_bf16_B%d_H64" % B
+    s.H = 64
+    s.scale = 1.0 / math.sqrt(256.0)
+    return s
+
+
 def profile_decode(B=8, L=65536, seed=0x5EED + 5) -> Spec:
     """bf16 decode, batch B at context L: a profiling case larger than L2 (0.75 GB resident)."""
     return Spec("profile_decode_bf16_B%d_L%d" % (B, L), lens=[L] * B, q_req=list(range(B)),
@@ -306,6 +317,7 @@ WORKLOADS = {
     "indexshare": indexshare,
     "prefill_q8": prefill_q8,
     "long_decode_q8": long_decode_q8,
+    "glm5_decode": glm5_decode,
     "profile_decode": profile_decode,
     "profile_prefill": profile_prefill,
     "profile_long": profile_long,

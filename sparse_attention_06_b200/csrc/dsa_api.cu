@@ -150,8 +150,8 @@ bool current_device_sms(int* num_sms) {
 MlaPlan mla_plan(bool decode, const void* q, int32_t q_dtype, int32_t H, int32_t d_v, int32_t d_rope,
                  const dsa_paged_cache& latent, int32_t T, int32_t k, const void* out, int num_sms) {
   MlaPlan pl{false, 1, 0};
-  pl.tensor_cores = H == 128 && d_v == 512 && d_rope == 64 && q_dtype == DSA_BF16 && latent.block_size == 64 &&
-                    aligned16(q) && aligned16(out) && aligned16(latent.data);
+  pl.tensor_cores = (H == 128 || H == 64) && d_v == 512 && d_rope == 64 && q_dtype == DSA_BF16 &&
+                    latent.block_size == 64 && aligned16(q) && aligned16(out) && aligned16(latent.data);
   if (pl.tensor_cores && T > 0) {
     pl.nsplit = decode ? mla_tc_num_splits(T, k, num_sms) : 1;
     pl.workspace_bytes = mla_tc_workspace_bytes(T, H, d_v, pl.nsplit);
@@ -387,7 +387,7 @@ dsa_status dsa_selftest_bounded_wait(int64_t limit_cycles, dsa_stream stream) {
 }
 
 size_t dsa_mla_workspace_size(int32_t num_queries, int32_t H, int32_t d_v, int32_t k) {
-  if (num_queries <= 0 || H != 128 || d_v != 512 || k < 1) return 0;
+  if (num_queries <= 0 || (H != 128 && H != 64) || d_v != 512 || k < 1) return 0;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   return mla_tc_workspace_bytes(num_queries, H, d_v, mla_tc_num_splits(num_queries, k, sms));

@@ -1,14 +1,16 @@
 // mla_tc.cu -- sparse MLA (MQA mode) over the selected latent rows on tcgen05 tensor cores.
 //
 // Page "How GLM5.3 Sparse Attention Affects HBM Memory Usage", sections "Sparse MLA" and "MLA
-// Modifications": all 128 heads share each selected 576-wide latent row (512 latent + 64 RoPE);
-// the logits are P = Q[H, 576] K^T over the selected rows and the output is O = softmax(P) V,
-// where V is the first 512 dims of the same rows.  The softmax is the usual scaled one.
+// Modifications": all H heads (128, or GLM-5's 64) share each selected 576-wide latent row (512
+// latent + 64 RoPE); the logits are P = Q[H, 576] K^T over the selected rows and the output is
+// O = softmax(P) V, where V is the first 512 dims of the same rows.  The softmax is the usual
+// scaled one.
 //
 // Work unit = (query t, key split sp, value half v).  A unit computes, for its slice of the
-// query's selected rows (64-row tiles), S = Q K^T on the tensor cores (M = 128 heads, N = 64 rows,
-// K = 576), an online softmax per head row, and O_v += P V_v (M = 128 heads, N = 256 value dims,
-// K = 64 rows) into tensor memory.  The full O (512 f32 columns) would fill tensor memory, so the
+// query's selected rows (64-row tiles), S = Q K^T on the tensor cores (M = H heads, N = 64 rows,
+// K = 576), an online softmax per head row, and O_v += P V_v (M = H heads, N = 256 value dims,
+// K = 64 rows) into tensor memory.  With M = 64 the products use lanes 0..15 of each 32-lane
+// tensor-memory quarter (GLM-5 shape; every other place is the same).  The full O (512 f32 columns) would fill tensor memory, so the
 // two value halves run on two CTAs, each recomputing S.
 // Tensor memory (512 columns): O_v [0, 256), S [256, 320), and the first 384 dims of Q
 // [320, 512) -- the S products read those as the A operand straight from tensor memory, so only
@@ -45,7 +47,6 @@ namespace dsa {
 namespace {
 
 
-constexpr int kH = 128;         // heads (MMA M)
 constexpr int kDqk = 576;       // latent + rope
 constexpr int kDv = 512;        // value dims
 constexpr int kHalf = 256;      // value dims per CTA
@@ -59,26 +60,34 @@ constexpr int kKeysPerWarp = kTile / kGatherWarps;  // 16
 constexpr int kPvWarp = kGatherWarps + 5;                 // issues the P V products
 constexpr int kThreads = 32 * (kGatherWarps + 1 + 4 + 1);
 
-constexpr int Q_CHUNK = kH * 128;                            // 16 KB: 128 head rows x 64 dims
-constexpr int QS_BYTES = (kChunks - kTmemQChunks) * Q_CHUNK; // 48 KB of Q in shared memory
 constexpr int K_CHUNK = kTile * 128;                         // 8 KB: 64 rows x 64 dims
 constexpr int K_BYTES = kChunks * K_CHUNK;                   // 72 KB
-constexpr int P_BYTES = kH * kTile * 2;                      // 16 KB
-constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + QS_BYTES;
-constexpr int OFF_P = OFF_K + kStages * K_BYTES;
-constexpr int OFF_BAR = OFF_P + P_BYTES;
 constexpr int NBAR = 2 + 3 * kStages + 8;
-constexpr int OFF_MASK = OFF_BAR + NBAR * 8;                 // valid-row masks [stage][gather warp]
-constexpr int OFF_MISC = OFF_MASK + kStages * kGatherWarps * 4;
-constexpr int OFF_STATS = OFF_MISC + 32;                    // 1 / l of each head row (last unit)
-constexpr int BYTES = OFF_STATS + kH * 4;
-constexpr int SMEM = BYTES + 1024;
-static_assert(SMEM <= 232448, "shared memory budget");
-
 constexpr int kQStaged = 5;                                  // staged Q: 64-dim boxes through shared memory
-static_assert(kQStaged == 4 + 1 && 4 * Q_CHUNK <= K_BYTES && Q_CHUNK == P_BYTES, "staging: 4 boxes in ring stage 1, 1 in P");
 static_assert(kQStaged + 1 == kTmemQChunks, "the last tensor-memory Q box is loaded directly");
+
+// Shapes that depend on the head count H (the MMA M: 128, or 64 for the GLM-5 shape).  With
+// M = 64 a product's rows sit in lanes 0..15 of each 32-lane tensor-memory quarter (row m in lane
+// 32 (m / 16) + m % 16), so a warp owns RQ = H / 4 head rows of its quarter: lanes 0..RQ-1.
+template <int H>
+struct HCfg {
+  static_assert(H == 64 || H == 128, "tensor-core MLA heads");
+  static constexpr int RQ = H / 4;                              // head rows per lane quarter
+  static constexpr int Q_CHUNK = H * 128;                       // H head rows x 64 dims
+  static constexpr int QS_BYTES = (kChunks - kTmemQChunks) * Q_CHUNK;  // Q in shared memory
+  static constexpr int P_BYTES = H * kTile * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + QS_BYTES;
+  static constexpr int OFF_P = OFF_K + kStages * K_BYTES;
+  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int OFF_MASK = OFF_BAR + NBAR * 8;         // valid-row masks [stage][gather warp]
+  static constexpr int OFF_MISC = OFF_MASK + kStages * kGatherWarps * 4;
+  static constexpr int OFF_STATS = OFF_MISC + 32;             // 1 / l of each head row (last unit)
+  static constexpr int BYTES = OFF_STATS + H * 4;
+  static constexpr int SMEM = BYTES + 1024;
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(4 * Q_CHUNK <= K_BYTES && Q_CHUNK == P_BYTES, "staging: 4 boxes in ring stage 1, 1 in P");
+};
 
 constexpr uint32_t TM_O = 0;       // O half: columns [0, 256)
 constexpr uint32_t TM_S = 256;     // S: [256, 320)
@@ -87,15 +96,15 @@ constexpr uint32_t TM_COLS = 512;
 
 struct Params {
   const __nv_bfloat16* latent;   // pool rows of 576
-  const __nv_bfloat16* q;        // [T, 128, 576]
+  const __nv_bfloat16* q;        // [T, H, 576]
   const int32_t* idx;
   const int32_t* q_req;
   const int32_t* q_pos;
   const int32_t* block_table;
-  __nv_bfloat16* out;            // [T, 128, 512] (single split)
-  float* lse;                    // [T, 128] or null (single split)
-  float* part_o;                 // [T, nsplit, 128, 512] (several splits)
-  float* part_lse;               // [T, nsplit, 128]
+  __nv_bfloat16* out;            // [T, H, 512] (single split)
+  float* lse;                    // [T, H] or null (single split)
+  float* part_o;                 // [T, nsplit, H, 512] (several splits)
+  float* part_lse;               // [T, nsplit, H]
   int64_t num_blocks;
   int32_t oob_row;               // first row past the pool (gathered as zeros)
   int T, k, ks, nsplit, num_reqs, max_blocks, max_context;
@@ -148,17 +157,20 @@ __device__ __forceinline__ int pos_block(const Params& p, bool qok, int req, int
   return blk;
 }
 
-// Pull the 128 x 576 query block of query t into L2 ahead of its use (16 KB pieces).
+// Pull the H x 576 query block of query t into L2 ahead of its use (16 KB pieces).
+template <int H>
 __device__ __forceinline__ void prefetch_q(const Params& p, int t) {
-  const uint8_t* src = reinterpret_cast<const uint8_t*>(p.q + (int64_t)t * kH * kDqk);
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(p.q + (int64_t)t * H * kDqk);
 #pragma unroll 1
-  for (int off = 0; off < kH * kDqk * 2; off += 16384) prefetch_l2_bulk(src + off, 16384u);
+  for (int off = 0; off < H * kDqk * 2; off += 16384) prefetch_l2_bulk(src + off, 16384u);
 }
 
-// Staging place of the staged Q's box c (dims [64 c, 64 c + 64), 128 rows, 128B-swizzled,
+// Staging place of the staged Q's box c (dims [64 c, 64 c + 64), H rows, 128B-swizzled,
 // 1024-byte aligned): boxes 0..3 in ring stage 1, box 4 in the P buffer.
+template <int H>
 __device__ __forceinline__ uint8_t* q_stage_box(uint8_t* smem, int c) {
-  return c < 4 ? smem + OFF_K + K_BYTES + c * Q_CHUNK : smem + OFF_P;
+  using HC = HCfg<H>;
+  return c < 4 ? smem + HC::OFF_K + K_BYTES + c * HC::Q_CHUNK : smem + HC::OFF_P;
 }
 
 // 64-row tiles of unit (t, sp): its split's share of the k selection slots, or, without a
@@ -170,28 +182,33 @@ __device__ __forceinline__ int unit_tiles(const Params& p, int t, int sp) {
   return n > 0 ? (n + kTile - 1) / kTile : 0;
 }
 
-// Rows [32 q, 32 q + 32) of O_v / l (q = this warp's tensor-memory lane quarter), columns
-// [c_lo, c_hi) of the value half (multiples of 64), from tensor memory to the partials (f32, with
-// key splits) or the output (bf16), through a 4 KB staging area: lane i stages its row i (128
-// bytes per block, 16-byte pieces XOR-permuted by i mod 8), then the warp writes rows 4k + lane/8,
-// piece lane mod 8, so that each global store instruction writes four whole 128-byte row pieces.
-// prow / orow: this lane's partial / output row.  have_o false (a unit without rows) stores zeros.
+// The RQ head rows of this warp's tensor-memory lane quarter (lanes 0..RQ-1), columns [c_lo,
+// c_hi) of O_v / l (multiples of 64), from tensor memory to the partials (f32, with key splits) or
+// the output (bf16), through a 4 KB staging area: lane i stages its row (128 bytes per block,
+// 16-byte pieces XOR-permuted by i mod 8), then the warp writes rows 4k + lane/8, piece lane mod
+// 8, so that each global store instruction writes four whole 128-byte row pieces (lanes past RQ
+// stage nothing that is written).  prow / orow: this lane's partial / output row (rows of a
+// quarter are consecutive).  have_o false (a unit without rows) stores zeros.
+template <int H>
 __device__ __forceinline__ void store_o(const Params& p, uint32_t lane_base, int c_lo, int c_hi, uint8_t* stage,
                                         float inv, bool have_o, int64_t prow, int64_t orow, int v) {
+  constexpr int RQ = HCfg<H>::RQ;
   const int lane = threadIdx.x & 31;
   const int srow = lane >> 3, spiece = lane & 7;
   const bool f32out = p.nsplit > 1;
+  // partial / output row of the quarter's first head row (every lane's r is that plus lane % RQ)
+  const int64_t prow0 = prow - lane % RQ, orow0 = orow - lane % RQ;
   // write the staged 128-byte block of each of this warp's rows to columns [col, col + 128 B)
   auto flush = [&](int col) {
     __syncwarp();
 #pragma unroll
-    for (int k4 = 0; k4 < 8; ++k4) {
-      const int rr = k4 * 4 + srow;  // row within this warp's 32
+    for (int k4 = 0; k4 < HCfg<H>::RQ / 4; ++k4) {
+      const int rr = k4 * 4 + srow;  // row within this warp's RQ
       const uint4 x = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((spiece ^ (rr & 7)) << 4));
       if (f32out)
-        *reinterpret_cast<uint4*>(p.part_o + (prow - lane + rr) * kDv + v * kHalf + col + spiece * 4) = x;
+        *reinterpret_cast<uint4*>(p.part_o + (prow0 + rr) * kDv + v * kHalf + col + spiece * 4) = x;
       else
-        *reinterpret_cast<uint4*>(p.out + (orow - lane + rr) * kDv + v * kHalf + col + spiece * 8) = x;
+        *reinterpret_cast<uint4*>(p.out + (orow0 + rr) * kDv + v * kHalf + col + spiece * 8) = x;
     }
     __syncwarp();
   };
@@ -208,7 +225,7 @@ __device__ __forceinline__ void store_o(const Params& p, uint32_t lane_base, int
 #pragma unroll
       for (int c = 0; c < 64; ++c) o[c] = 0u;
     }
-    uint8_t* srow_ptr = stage + lane * 128;
+    uint8_t* srow_ptr = stage + lane * 128;  // (staged only by lanes 0..RQ-1: RQ * 128 bytes)
     if (f32out) {
       // two blocks of 32 f32 columns
 #pragma unroll
@@ -216,9 +233,10 @@ __device__ __forceinline__ void store_o(const Params& p, uint32_t lane_base, int
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int c = 32 * b + 4 * j;
-          *reinterpret_cast<float4*>(srow_ptr + ((j ^ (lane & 7)) << 4)) =
-              make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
-                          __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
+          if (lane < RQ)
+            *reinterpret_cast<float4*>(srow_ptr + ((j ^ (lane & 7)) << 4)) =
+                make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
+                            __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
         }
         flush(c0 + 32 * b);
       }
@@ -233,23 +251,27 @@ __device__ __forceinline__ void store_o(const Params& p, uint32_t lane_base, int
                                                           __uint_as_float(o[8 * j + 2 * e + 1]) * inv);
           pk[e] = *reinterpret_cast<const uint32_t*>(&hv);
         }
-        *reinterpret_cast<uint4*>(srow_ptr + ((j ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        if (lane < RQ) *reinterpret_cast<uint4*>(srow_ptr + ((j ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       flush(c0);
     }
   }
 }
 
-template <bool kStagedQ>
+template <int H, bool kStagedQ>
 __global__ void __launch_bounds__(kThreads, 1)
     mla_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap lmap,
                   const Params p) {
+  using HC = HCfg<H>;
+  constexpr int RQ = HC::RQ;
+  constexpr int Q_CHUNK = HC::Q_CHUNK;
+  constexpr int QS_BYTES = HC::QS_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_s = smem + OFF_Q;
-  uint8_t* k_ring = smem + OFF_K;
-  uint8_t* p_s = smem + OFF_P;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint8_t* q_s = smem + HC::OFF_Q;
+  uint8_t* k_ring = smem + HC::OFF_K;
+  uint8_t* p_s = smem + HC::OFF_P;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + HC::OFF_BAR);
   uint64_t* q_full = bars + 0;                 // Q of the unit in place (TMEM part + smem part)
   uint64_t* q_empty = bars + 1;                // the unit's last Q K^T has completed
   uint64_t* k_full = bars + 2;                 // [kStages] rows landed
@@ -263,10 +285,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_first = mma_fin + 1;             // staged Q: all of it in place
   uint64_t* q_stage = q_first + 1;             // staged Q: dims [0, 320) in shared memory
   uint64_t* ep_half = q_stage + 1;             // last unit: row statistics published after its last P V
-  float* stats = reinterpret_cast<float*>(smem + OFF_STATS);
-  uint32_t* masks = reinterpret_cast<uint32_t*>(smem + OFF_MASK);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 8);
+  float* stats = reinterpret_cast<float*>(smem + HC::OFF_STATS);
+  uint32_t* masks = reinterpret_cast<uint32_t*>(smem + HC::OFF_MASK);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + HC::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + HC::OFF_MISC + 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int units = p.T * p.nsplit * 2;
@@ -280,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (blockIdx.x < units) {
       int t0, sp0, v0;
       unit_coords(p, blockIdx.x, t0, sp0, v0);
-      prefetch_q(p, t0);
+      prefetch_q<H>(p, t0);
     }
     mbar_init(q_full, 32 * kGatherWarps + 1);
     mbar_init(q_empty, 1);
@@ -312,8 +334,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < kGatherWarps) {
     // ------------------------------------------------------------------ Q and row gather
-    const int gw = warp;                  // keys gw*16 .. gw*16+15 of each tile; head rows gw*32..
-    const int h = gw * 32 + lane;
+    const int gw = warp;                  // keys gw*16 .. gw*16+15 of each tile; head rows gw*RQ..
+    // this lane's head row (lanes past RQ, which hold no row with H = 64, repeat one: they fill
+    // tensor-memory lanes no product reads)
+    const int h = gw * RQ + (lane % RQ);
     const uint32_t my_lanes = tmem + ((uint32_t)(gw * 32) << 16);
     int gi = 0;  // CTA-wide tile counter
     int ui = 0;  // CTA-wide unit counter
@@ -324,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (gw == 0 && lane == 0 && u + (int)gridDim.x < units) {
         int tn, spn, vn;
         unit_coords(p, u + gridDim.x, tn, spn, vn);
-        if (tn != t) prefetch_q(p, tn);  // the next unit's queries, while this one runs
+        if (tn != t) prefetch_q<H>(p, tn);  // the next unit's queries, while this one runs
       }
       // Row lookups of this warp's 16 keys per tile (lanes 0..15), software-pipelined so that no
       // load is waited on in the tile it is issued: the selected position two tiles ahead and the
@@ -346,9 +370,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (gw == 0 && lane == 0) {
           mbar_arrive_expect_tx(q_full, QS_BYTES);
           for (int c = kTmemQChunks; c < kChunks; ++c)
-            tma_load_2d(q_s + (c - kTmemQChunks) * Q_CHUNK, &qmap, q_full, c * 64, t * kH);
+            tma_load_2d(q_s + (c - kTmemQChunks) * Q_CHUNK, &qmap, q_full, c * 64, t * H);
         }
-        const uint4* src = reinterpret_cast<const uint4*>(p.q + ((int64_t)t * kH + h) * kDqk);
+        const uint4* src = reinterpret_cast<const uint4*>(p.q + ((int64_t)t * H + h) * kDqk);
 #pragma unroll 1
         for (int b = 0; b < 2; ++b) {  // 192 dims = 96 columns per batch, all loads in flight
           uint32_t w[96];
@@ -412,9 +436,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // 1 / l (after the unit's last P V, which also frees the row ring for the staging)
         if (!(ok = warp_wait(ep_half, 0, p.err, abort_flag))) break;
         tc_fence_after();
-        const int64_t orow = (int64_t)t * kH + h;
-        const int64_t prow = ((int64_t)t * p.nsplit + sp) * kH + h;
-        store_o(p, my_lanes, kHalf / 2, kHalf, k_ring + gw * 4096, stats[h], ntiles > 0, prow, orow, v);
+        const int64_t orow = (int64_t)t * H + h;
+        const int64_t prow = ((int64_t)t * p.nsplit + sp) * H + h;
+        store_o<H>(p, my_lanes, kHalf / 2, kHalf, k_ring + gw * RQ * 128, stats[h], ntiles > 0, prow, orow, v);
         tc_fence_before();
       }
     }
@@ -426,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kGatherWarps) {
     // ------------------------------------------------------------------ Q K^T issuer
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_f16(1u, 0u, 128u, (uint32_t)kTile);  // S: B K-major
+      const uint32_t idesc_s = idesc_f16(1u, 0u, (uint32_t)H, (uint32_t)kTile);  // S: B K-major
       int gi = 0, ui = 0;
       bool ok = true;
       const uint64_t qd = sw128_desc(smem_u32(q_s), 16, 1024);
@@ -477,12 +501,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         unit_coords(p, blockIdx.x, t0, sp0, v0);
         mbar_arrive_expect_tx(q_first, QS_BYTES);
         for (int c = kTmemQChunks; c < kChunks; ++c)
-          tma_load_2d(q_s + (c - kTmemQChunks) * Q_CHUNK, &qmap, q_first, c * 64, t0 * kH);
+          tma_load_2d(q_s + (c - kTmemQChunks) * Q_CHUNK, &qmap, q_first, c * 64, t0 * H);
         mbar_arrive_expect_tx(q_stage, kQStaged * Q_CHUNK);
         for (int c = 0; c < kQStaged; ++c)
-          tma_load_2d(q_stage_box(smem, c), &qmap, q_stage, c * 64, t0 * kH);
+          tma_load_2d(q_stage_box<H>(smem, c), &qmap, q_stage, c * 64, t0 * H);
       }
-      const uint32_t idesc_o = idesc_f16(1u, 1u, 128u, (uint32_t)kHalf);  // O: B (V) MN-major
+      const uint32_t idesc_o = idesc_f16(1u, 1u, (uint32_t)H, (uint32_t)kHalf);  // O: B (V) MN-major
       // P [128 x 64] K-major, no swizzle: 8x16-byte core matrices 128 B apart along K and 1024 B
       // apart along M; one K step (16 keys) is two core matrices = 256 bytes
       const uint64_t pd = noswz_desc(smem_u32(p_s), 128, 1024);
@@ -518,7 +542,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < kPvWarp) {
     // ------------------------------------------------------------------ softmax + epilogue
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;  // head row
+    // this lane's head row; with H = 64 lanes RQ..31 of the quarter hold no row: they see every
+    // key as masked and write nothing (their r repeats a row only to keep addresses in range)
+    const bool row_lane = lane < RQ;
+    const int r = quarter * RQ + (lane % RQ);
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     if constexpr (staged_q) {
       // the staged Q, head row r, dims [0, 384) into tensor-memory columns [320, 512): dims
@@ -526,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // j ^ (r mod 8)), dims [320, 384) straight from global memory
       int t0, sp0, v0;
       unit_coords(p, blockIdx.x, t0, sp0, v0);
-      const uint4* src = reinterpret_cast<const uint4*>(p.q + ((int64_t)t0 * kH + r) * kDqk) + 5 * 8;
+      const uint4* src = reinterpret_cast<const uint4*>(p.q + ((int64_t)t0 * H + r) * kDqk) + 5 * 8;
       uint32_t w[32];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -536,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool qs_ok = mbar_wait(q_stage, 0, p.err, abort_flag);
 #pragma unroll 1
       for (int c = 0; c < kQStaged && qs_ok; ++c) {
-        const uint8_t* row = q_stage_box(smem, c) + r * 128;
+        const uint8_t* row = q_stage_box<H>(smem, c) + r * 128;
         uint32_t x[32];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -576,6 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint64_t valid = 0u;
 #pragma unroll
         for (int w = 0; w < kGatherWarps; ++w) valid |= (uint64_t)masks[s * kGatherWarps + w] << (w * kKeysPerWarp);
+        if (!row_lane) valid = 0u;
         float mt = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
@@ -628,10 +656,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         l += psum;
         // P row r: 8 core-matrix rows of 16 B (8 keys each), no swizzle
-        uint8_t* prow = p_s + (r >> 3) * 1024 + (r & 7) * 16;
+        if (row_lane) {
+          uint8_t* prow = p_s + (r >> 3) * 1024 + (r & 7) * 16;
 #pragma unroll
-        for (int kc = 0; kc < 8; ++kc)
-          *reinterpret_cast<uint4*>(prow + kc * 128) = make_uint4(pk[4 * kc], pk[4 * kc + 1], pk[4 * kc + 2], pk[4 * kc + 3]);
+          for (int kc = 0; kc < 8; ++kc)
+            *reinterpret_cast<uint4*>(prow + kc * 128) = make_uint4(pk[4 * kc], pk[4 * kc + 1], pk[4 * kc + 2], pk[4 * kc + 3]);
+        }
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(p_full);
@@ -643,18 +673,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv = l > 0.0f ? 1.0f / l : 0.0f;
       const float lse = l > 0.0f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
-      const int64_t orow = (int64_t)t * kH + r;
-      const int64_t prow = ((int64_t)t * p.nsplit + sp) * kH + r;
-      // O / l leaves through this warp's 4 KB quarter of the P buffer (free: the last P V has
-      // completed).  In the CTA's last unit the gather warps, idle by then, store the columns
+      const int64_t orow = (int64_t)t * H + r;
+      const int64_t prow = ((int64_t)t * p.nsplit + sp) * H + r;
+      // O / l leaves through this warp's quarter of the P buffer (RQ * 128 bytes; free: the last
+      // P V has completed).  In the CTA's last unit the gather warps, idle by then, store the columns
       // [128, 256) of the half: they get 1 / l through shared memory once the last P V is done.
       const bool last = u + (int)gridDim.x >= units;
       if (last) {
-        stats[r] = inv;
+        if (row_lane) stats[r] = inv;
         mbar_arrive(ep_half);
       }
-      store_o(p, lane_base, 0, last ? kHalf / 2 : kHalf, p_s + quarter * 4096, inv, ntiles > 0, prow, orow, v);
-      if (v == 0) {
+      store_o<H>(p, lane_base, 0, last ? kHalf / 2 : kHalf, p_s + quarter * RQ * 128, inv, ntiles > 0, prow, orow, v);
+      if (v == 0 && row_lane) {
         if (p.nsplit == 1) {
           if (p.lse) p.lse[orow] = lse;
         } else {
@@ -673,12 +703,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// grid (T, 128 heads), block 256: merge the split partials of one (query, head) row.  The split
+// grid (T, H heads), block 256: merge the split partials of one (query, head) row.  The split
 // weights exp(LSE_sp - max) go to shared memory first; then thread i sums column group i % 128
 // (4 of the 512 value columns) over the splits i / 128, i / 128 + 2, ... with up to 16 loads in
 // flight, and the two halves are added through shared memory.
 constexpr int kMaxSplits = 64;
 constexpr int kCombThreads = 256;
+template <int H>
 __global__ void __launch_bounds__(kCombThreads) mla_combine_kernel(const float* __restrict__ part_o,
                                                                    const float* __restrict__ part_lse, int nsplit,
                                                                    __nv_bfloat16* __restrict__ out,
@@ -690,14 +721,14 @@ __global__ void __launch_bounds__(kCombThreads) mla_combine_kernel(const float* 
   const int c4 = threadIdx.x & 127, half = threadIdx.x >> 7;
   griddep_launch_dependents();
   griddep_wait();  // the partials come from the kernel before
-  const int64_t row0 = (int64_t)t * nsplit * kH + h;  // partial row of split 0; split sp adds sp*kH
+  const int64_t row0 = (int64_t)t * nsplit * H + h;  // partial row of split 0; split sp adds sp*H
   if (threadIdx.x < 32) {
     float mx = -INFINITY;
-    for (int sp = threadIdx.x; sp < nsplit; sp += 32) mx = fmaxf(mx, part_lse[row0 + (int64_t)sp * kH]);
+    for (int sp = threadIdx.x; sp < nsplit; sp += 32) mx = fmaxf(mx, part_lse[row0 + (int64_t)sp * H]);
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
     float sum = 0.0f;
     for (int sp = threadIdx.x; sp < nsplit; sp += 32) {
-      const float ls = part_lse[row0 + (int64_t)sp * kH];
+      const float ls = part_lse[row0 + (int64_t)sp * H];
       const float wgt = ls == -INFINITY ? 0.0f : expf(ls - mx);
       wts[sp] = wgt;
       sum += wgt;
@@ -711,7 +742,7 @@ __global__ void __launch_bounds__(kCombThreads) mla_combine_kernel(const float* 
   __syncthreads();
   float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   const float4* src = reinterpret_cast<const float4*>(part_o + row0 * kDv) + c4;
-  const int64_t step = (int64_t)kH * kDv / 4;  // float4s from one split's row to the next
+  const int64_t step = (int64_t)H * kDv / 4;  // float4s from one split's row to the next
   for (int sp0 = half; sp0 < nsplit; sp0 += 32) {
     float4 a[16];
 #pragma unroll
@@ -739,8 +770,8 @@ __global__ void __launch_bounds__(kCombThreads) mla_combine_kernel(const float* 
     uint2 pk;
     pk.x = *reinterpret_cast<const uint32_t*>(&lo);
     pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(out + ((int64_t)t * kH + h) * kDv + 4 * c4) = pk;
-    if (lse_out && threadIdx.x == 0) lse_out[(int64_t)t * kH + h] = s_lse;
+    *reinterpret_cast<uint2*>(out + ((int64_t)t * H + h) * kDv + 4 * c4) = pk;
+    if (lse_out && threadIdx.x == 0) lse_out[(int64_t)t * H + h] = s_lse;
   }
 }
 
@@ -780,10 +811,14 @@ size_t mla_tc_workspace_bytes(int T, int H, int d_v, int nsplit) {
   return ((o + 255) / 256) * 256 + ((l + 255) / 256) * 256;
 }
 
-cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_t s) {
+namespace {
+
+template <int H>
+cudaError_t launch_mla_tc_h(const MlaArgs& a, int nsplit, int num_sms, cudaStream_t s) {
+  using HC = HCfg<H>;
   const int T = a.batch.num_queries;
   alignas(64) CUtensorMap qmap, lmap;
-  if (!encode_tmap_2d(&qmap, a.q, 2, kDqk, (uint64_t)T * kH, kDqk * 2, 64, kH, true)) return cudaErrorInvalidValue;
+  if (!encode_tmap_2d(&qmap, a.q, 2, kDqk, (uint64_t)T * H, kDqk * 2, 64, H, true)) return cudaErrorInvalidValue;
   const uint64_t pool_rows = (uint64_t)a.latent.num_blocks * kPage;
   if (pool_rows >= 0x7FFFFFFFull) return cudaErrorInvalidValue;  // row coordinates are 32-bit
   if (!encode_tmap_2d(&lmap, a.latent.data, 2, kDqk, pool_rows, (uint64_t)kDqk * 2, 64, 1, true))
@@ -812,23 +847,29 @@ cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_
   p.part_o = nullptr;
   p.part_lse = nullptr;
   if (nsplit > 1) {
-    const size_t o = (size_t)T * nsplit * kH * kDv * sizeof(float);
+    const size_t o = (size_t)T * nsplit * H * kDv * sizeof(float);
     p.part_o = static_cast<float*>(a.workspace);
     p.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) + ((o + 255) / 256) * 256);
   }
   const int units = T * nsplit * 2;
   const int grid = units < num_sms ? units : num_sms;
-  auto kernel = units <= grid ? mla_tc_kernel<true> : mla_tc_kernel<false>;  // one unit per CTA: staged Q
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  auto kernel = units <= grid ? mla_tc_kernel<H, true> : mla_tc_kernel<H, false>;  // one unit per CTA: staged Q
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HC::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attrs[2];
-  const cudaLaunchConfig_t cfg = launch_config(dim3(grid), dim3(kThreads), SMEM, s, attrs);
+  const cudaLaunchConfig_t cfg = launch_config(dim3(grid), dim3(kThreads), HC::SMEM, s, attrs);
   e = cudaLaunchKernelEx(&cfg, kernel, qmap, lmap, p);
   if (e != cudaSuccess || nsplit == 1) return e;
   cudaLaunchAttribute cattrs[2];
-  const cudaLaunchConfig_t ccfg = launch_config(dim3(T, kH), dim3(kCombThreads), 0, s, cattrs);
-  return cudaLaunchKernelEx(&ccfg, mla_combine_kernel, (const float*)p.part_o, (const float*)p.part_lse, nsplit, p.out,
-                            a.lse);
+  const cudaLaunchConfig_t ccfg = launch_config(dim3(T, H), dim3(kCombThreads), 0, s, cattrs);
+  return cudaLaunchKernelEx(&ccfg, mla_combine_kernel<H>, (const float*)p.part_o, (const float*)p.part_lse, nsplit,
+                            p.out, a.lse);
+}
+
+}  // namespace
+
+cudaError_t launch_mla_tc(const MlaArgs& a, int nsplit, int num_sms, cudaStream_t s) {
+  return a.H == 64 ? launch_mla_tc_h<64>(a, nsplit, num_sms, s) : launch_mla_tc_h<128>(a, nsplit, num_sms, s);
 }
 
 }  // namespace dsa

@@ -23,10 +23,9 @@
 //      positions take every score (no threshold).  A histogram that does not describe the row
 //      (one left dirty) only leads to a wrong tau, which step 2's count catches (exact path).
 //      Each CTA clears its share of the histogram row once every CTA has used it.
-//   2. Filter.  One coalesced pass over the slice, two batches of 4096 scores in flight ahead of
-//      the one it filters, appends every (key, position) with score >= tau to shared memory (one
-//      shared atomic per warp and 256 scores), and the CTA stores its candidate count into every
-//      CTA of the cluster.
+//   2. Filter.  One coalesced pass over the slice appends every (key, position) with
+//      score >= tau to shared memory (one shared atomic per warp and 512 scores), and the CTA
+//      stores its candidate count into every CTA of the cluster.
 //   3. Exact K-th key.  After a cluster barrier every CTA gathers all candidate keys of the row
 //      through distributed shared memory and radix-selects the K-th largest key Tk among them.
 //      If the row had at least K candidates, every score >= Tk is a candidate, so Tk is the
@@ -61,8 +60,7 @@ constexpr int kMaxSlice = 1 << 17;         // positions one CTA's bitmap covers
 constexpr int kMaxCluster = 8;
 constexpr int kSample = 4096;              // sampled keys (512 chunks of 8)
 constexpr int kPer = 16;                   // scores per thread per step of the exact path
-constexpr int kFPer = 8;                   // scores per thread per filter batch
-constexpr int kFStep = kFPer * kThreads;   // scores per filter batch
+constexpr int kFPer = 16;                  // scores per thread per filter batch
 static_assert(kHBins == 8 * kThreads, "each thread scans 8 histogram bins");
 static_assert(kCap >= kSample, "the sample fits the key pool");
 static_assert(kKeyBins == 8 * kThreads, "each thread reads 8 bins of a digit histogram row");
@@ -471,11 +469,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int words = (len + 31) >> 5;
   const float* srow = row + lo;
   const bool vec = ((reinterpret_cast<uintptr_t>(srow) & 15u) == 0);
-  // the filter below keeps two batches of loads in flight ahead of the one it processes; the
-  // first two are issued now, so that they land during step 1
-  float v0[kFPer], v1[kFPer], v2[kFPer];
-  load_batch(srow, len, 0, vec, v0);
-  load_batch(srow, len, kFStep, vec, v1);
+  constexpr int kStep = kFPer * kThreads;
+  float v[kFPer];
+  load_batch(srow, len, 0, vec, v);  // the first batch of this slice, in flight during step 1
   for (int w = tid; w < words; w += kThreads) S.bitmap[w] = 0u;
   clear_hist(0);
   clear_hist(1);
@@ -510,6 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t p = (((int64_t)(s >> 3) * n / kChunks) & ~int64_t(7)) + (s & 7);
         sv[e] = row[p];
       }
+      // the first batch is consumed here (NaN check), so that its loads complete with the sample's
+      // rather than after step 1
+#pragma unroll
+      for (int j = 0; j < kFPer; ++j) saw_nan |= v[j] != v[j];
 #pragma unroll
       for (int e = 0; e < kSPT; ++e) S.pool[tid + e * kThreads] = order_key(sv[e], saw_nan);
       __syncthreads();  // sample keys and cleared histograms visible
@@ -522,11 +522,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();  // the counters are clear
   }
 
-  // 2. filter: append (key, position) of every score >= tau in this slice.  The three batch
-  //    registers take turns (no copies between them, which would wait for the loads in flight):
-  //    while one batch is filtered the next two are on their way.
-  auto filter_batch = [&](int base, float (&v)[kFPer], float (&ahead)[kFPer]) {
-    if (base + 2 * kFStep < len) load_batch(srow, len, base + 2 * kFStep, vec, ahead);
+  // 2. filter: append (key, position) of every score >= tau in this slice; the next batch's loads
+  //    are issued before the current batch is processed
+  for (int base = 0; base < len; base += kStep) {
+    float vn[kFPer];
+    if (base + kStep < len) load_batch(srow, len, base + kStep, vec, vn);
     uint32_t mask = 0u;
 #pragma unroll
     for (int j = 0; j < kFPer; ++j) {
@@ -550,11 +550,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         S.cand_pos[at] = (uint32_t)(lo + base + ((j >> 2) * kThreads + tid) * 4 + (j & 3));
       }
     }
-  };
-  for (int base = 0; base < len; base += 3 * kFStep) {
-    filter_batch(base, v0, v2);
-    if (base + kFStep < len) filter_batch(base + kFStep, v1, v0);
-    if (base + 2 * kFStep < len) filter_batch(base + 2 * kFStep, v2, v1);
+#pragma unroll
+    for (int j = 0; j < kFPer; ++j) v[j] = vn[j];
   }
   if (saw_nan) S.scal[4] = 1u;  // benign race: every writer stores 1
   __syncthreads();

@@ -109,7 +109,13 @@ def test_mla_split_plan_and_workspace(lib):
     assert lib.dsa_mla_workspace_size(64, 128, 512, 2048) == 0
     assert lib.dsa_mla_workspace_size(2, 128, 512, 100) == 0   # two tiles per query: no split
     assert lib.dsa_mla_workspace_size(0, 128, 512, 2048) == 0
-    assert lib.dsa_mla_workspace_size(4, 64, 512, 2048) == 0    # not the tensor-core shape
+    # the GLM-5 shape (64 heads) takes the same plan, with half the partial rows
+    def ws64(T, nsplit):
+        o = T * nsplit * 64 * 512 * 4
+        l = T * nsplit * 64 * 4
+        return ((o + 255) // 256) * 256 + ((l + 255) // 256) * 256
+    assert lib.dsa_mla_workspace_size(16, 64, 512, 2048) == ws64(16, 4)
+    assert lib.dsa_mla_workspace_size(4, 32, 512, 2048) == 0    # not a tensor-core shape
 
 
 def test_indexer_topk_workspace_size(lib):

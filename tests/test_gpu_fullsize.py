@@ -21,6 +21,9 @@ pytestmark = pytest.mark.gpu
     ("batched_decode", [0, 17, 38, 63], "bf16", "decode"),
     ("prefill", [0, 1, 2, 3, 1365, 2730, 4092, 4095], "e4m3", "prefill"),
     ("long_decode", [0, 9, 15], "e4m3", "decode"),
+    ("long_decode_q8", [0, 15], "e4m3", "decode"),
+    ("prefill_q8", [0, 2047, 4095], "e4m3", "prefill"),
+    ("glm5_decode", [0, 31, 63], "bf16", "decode"),
 ])
 def test_fullsize_sampled(name, queries, kind, entry):
     spec = di.WORKLOADS[name]()

@@ -427,3 +427,21 @@ def test_fused_indexer_topk_matches_unfused_and_reuses_workspace():
             assert int(ws.abs().sum()) == 0
         assert dsa.dsa_get_device_error() == 0
         check_topk(ref.cpu(), scores.cpu(), [L - 1 for L in spec.lens], spec.k)
+
+
+# ---------------------------------------------------------------------------------------------
+# the GLM-5 attention shape: 64 heads, softmax scale 1/sqrt(256)
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("lens,entry", [
+    ([6000], "decode"),                          # one query: 32 splits, one unit per CTA (staged Q)
+    ([3000, 2500, 7000, 300], "decode"),         # few queries: splits and the combine kernel
+    ([2100] * 80, "decode"),                     # more units than SMs: CTAs loop over units
+    ([3000, 2500, 7000, 300], "prefill"),        # whole queries per CTA
+])
+def test_glm5_shape_64_heads(lens, entry):
+    spec = di.Spec("glm5", lens=lens, q_req=list(range(len(lens))), q_pos=[L - 1 for L in lens], H=64,
+                   scale=1.0 / math.sqrt(256.0), seed=71)
+    x = to_dev(di.generate(spec, "cpu"))
+    queries = None if len(lens) < 10 else list(range(0, len(lens), 9))
+    parity_case(x, queries=queries, kind="bf16", mla_entry=entry)
