@@ -492,6 +492,19 @@ def run_cuda(args):
         breakdown["group_saving"] = 1.0 - ms_per_step / (n_l * fl_ms)
     err = dsa.dsa_get_device_error()
 
+    # the planted tail as the GPU's own scores show it (request 0): how far the median planted
+    # score sits above the unplanted scores' mean, in their standard deviations
+    planted = None
+    if spec.planted_frac > 0 and not layer.dense:
+        t0 = spec.q_req.index(0)
+        row = layer.scores[t0, :spec.q_pos[t0] + 1].double().cpu()
+        pos = di.planted_positions(spec, 0)
+        mask = torch.ones(row.numel(), dtype=torch.bool)
+        mask[pos] = False
+        unpl = row[mask]
+        planted = {"frac": spec.planted_frac, "beta": spec.planted_sigma,
+                   "lift_sigma_measured": float((row[pos].median() - unpl.mean()) / unpl.std())}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(x, spec, budget_s=args.cpu_budget)
@@ -508,6 +521,7 @@ def run_cuda(args):
                        "l2": ("inputs larger than L2: steps rotate over %d identical copies" % ncopy
                               if ncopy > 1 else "inputs larger than L2"),
                        "parallelism": "replicas x%d" % world},
+            "planted_tail": planted,
             "e2e": {"value": e2e_value, "unit": "query-tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h,
                     "note": "query-side inputs copied from pinned host memory every step; KV caches resident"},

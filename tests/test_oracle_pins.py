@@ -317,3 +317,28 @@ def test_indexer_e4m3_queries_dequantise_per_head():
     s_3 = oracle.indexer_scores(codes, x["w"], *args, q_scale=scale * 3.0)
     n = int(x["q_pos"][0]) + 1
     assert np.allclose(s_3[0, :n], 3.0 * s_q8[0, :n], rtol=1e-12, atol=0)
+
+
+def test_planted_tail_calibration():
+    # the long-context workload's planted keys are shifted by the beta that the committed
+    # calibration script found with this oracle; on its draw the median planted score sits
+    # 3 unplanted standard deviations above the unplanted mean
+    import importlib.util
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "make_planted_beta.py")
+    stored = json.load(open(os.path.join(os.path.dirname(path), "planted_beta.json")))
+    assert di.PLANTED_BETA == stored["beta"] and di.long_decode().planted_sigma == stored["beta"]
+    spec_ = importlib.util.spec_from_file_location("make_planted_beta", path)
+    mod = importlib.util.module_from_spec(spec_)
+    spec_.loader.exec_module(mod)
+    spec = di.long_decode(B=1)
+    q_idx, w, kraw, bt, _ = mod.draw_request(spec)
+    L = spec.lens[0]
+    rows = bt[0].long()[torch.arange(L) // di.BLOCK] * di.BLOCK + torch.arange(L) % di.BLOCK
+    base = kraw[rows]
+    planted = di.planted_positions(spec, 0)
+    mask = torch.ones(L, dtype=torch.bool)
+    mask[planted] = False
+    unpl = mod.scores_of(base, q_idx, w)[mask.numpy()]
+    got = mod.lift(stored["beta"], base, planted, di.plant_direction(q_idx[0], w[0]), q_idx, w,
+                   float(unpl.mean()), float(unpl.std()))
+    assert abs(got - 3.0) < 0.01
