@@ -654,7 +654,7 @@ def main(argv=None):
     ap.add_argument("--config", default="batched_decode",
                     choices=["tiny", "decode", "batched_decode", "prefill", "long_decode", "short_decode",
                              "indexshare", "prefill_q8", "long_decode_q8", "glm5_decode", "profile_decode",
-                             "profile_prefill", "profile_long"])
+                             "profile_prefill", "profile_long", "profile_long_q8"])
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -317,6 +317,14 @@ def profile_decode(B=8, L=65536, seed=0x5EED + 5) -> Spec:
                 q_pos=[L - 1] * B, seed=seed)
 
 
+def profile_long_q8(B=8, L=202752, seed=0x5EED + 7) -> Spec:
+    """Long-context decode at batch 8 with e4m3 indexer keys and queries, for profiling captures."""
+    s = profile_long(B, L, seed)
+    s.name = "profile_long_e4m3q_B%d_L%d" % (B, L)
+    s.q_idx_dtype = "e4m3"
+    return s
+
+
 def profile_prefill(ctx=16384, chunk=1024, seed=0x5EED + 6) -> Spec:
     """A smaller prefill chunk (e4m3 keys) for profiling captures."""
     return prefill(ctx=ctx, chunk=chunk, seed=seed)
@@ -342,6 +350,7 @@ WORKLOADS = {
     "profile_decode": profile_decode,
     "profile_prefill": profile_prefill,
     "profile_long": profile_long,
+    "profile_long_q8": profile_long_q8,
 }
 
 
