@@ -352,6 +352,13 @@ __device__ __noinline__ void topk_exact(const float* row, int64_t n, int k, int3
   }
 }
 
+// max(a, b), NaN when either is NaN
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
 // v[j] for a j known only at run time, without indexing the register array
 __device__ __forceinline__ float pick(const float (&v)[kFPer], int j) {
   float x = v[0];
@@ -523,18 +530,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // 2. filter: append (key, position) of every score >= tau in this slice; the next batch's loads
-  //    are issued before the current batch is processed
+  //    are issued before the current batch is processed.  Every score takes a comparison and a
+  //    NaN-propagating max (NaN in the slice <=> NaN max; load_batch gives 0 past the slice, and
+  //    only a last, partial batch tests positions).  With take_all the threshold is -inf: a NaN
+  //    score is then no candidate, which changes no result (its key is the lowest: it is selected
+  //    only when fewer than K other scores exist, and then the exact path below runs).
+  const float tau_eff = take_all ? -INFINITY : tau_f;
+  float nan_max = 0.0f;
   for (int base = 0; base < len; base += kStep) {
     float vn[kFPer];
     if (base + kStep < len) load_batch(srow, len, base + kStep, vec, vn);
     uint32_t mask = 0u;
+    if (base + kStep <= len) {
 #pragma unroll
-    for (int j = 0; j < kFPer; ++j) {
-      const int i = base + ((j >> 2) * kThreads + tid) * 4 + (j & 3);
-      const bool valid = i < len;
-      saw_nan |= valid && (v[j] != v[j]);
-      const bool pass = valid && (take_all || v[j] >= tau_f);
-      mask |= (uint32_t)pass << j;
+      for (int j = 0; j < kFPer; ++j) {
+        nan_max = max_nan(nan_max, v[j]);
+        mask |= (uint32_t)(v[j] >= tau_eff) << j;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kFPer; ++j) {
+        const int i = base + ((j >> 2) * kThreads + tid) * 4 + (j & 3);
+        nan_max = max_nan(nan_max, v[j]);
+        mask |= (uint32_t)(i < len && v[j] >= tau_eff) << j;
+      }
     }
     const uint32_t c = (uint32_t)__popc(mask);
     const uint32_t incl = warp_inclusive_scan(c);
@@ -553,6 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int j = 0; j < kFPer; ++j) v[j] = vn[j];
   }
+  saw_nan |= nan_max != nan_max;
   if (saw_nan) S.scal[4] = 1u;  // benign race: every writer stores 1
   __syncthreads();
   if (tid < (int)C) st_cluster_u32(&S.cnt_all[r], (uint32_t)tid, S.scal[5]);
