@@ -236,6 +236,7 @@ class Layer:
         import torch
         import sparse_attention_06_b200 as dsa
         self.dsa = dsa
+        self.torch = torch
         self.x = x
         spec = x["spec"]
         self.spec = spec
@@ -249,7 +250,19 @@ class Layer:
         self.idx = torch.empty((spec.T, spec.k), dtype=torch.int32, device=dev)
         self.out = torch.empty((spec.T, spec.H, spec.d_v), dtype=x["q_mla"].dtype, device=dev)
         self.lse = torch.empty((spec.T, spec.H), dtype=torch.float32, device=dev)
-        ws = dsa.dsa_mla_workspace_size(spec.T, spec.H, spec.d_v, spec.k)
+        # end to end, a large batch's MLA runs in query chunks, so that the output of one chunk goes
+        # back to the host while the next is computed: as many chunks (1, 2 or 4, whole query
+        # groups) as keep every chunk at four or more (query, value half) units per SM
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count if dev.type == "cuda" else 148
+        nch = next(c for c in (4, 2, 1) if c == 1 or 2 * spec.T // c >= 4 * sms)
+        g = max(1, spec.query_group)
+        cuts = sorted({min(spec.T, (spec.T * i // nch) // g * g) for i in range(nch + 1)})
+        self.chunks = [(c0, c1, dsa.Batch(x["q_req"][c0:c1], x["q_pos"][c0:c1], x["block_table"], self.max_ctx,
+                                          spec.query_group)) for c0, c1 in zip(cuts[:-1], cuts[1:]) if c1 > c0]
+        self.chunk_done = [torch.cuda.Event() for _ in self.chunks] if dev.type == "cuda" else []
+        self.back = torch.cuda.Event() if dev.type == "cuda" else None
+        ws = max(dsa.dsa_mla_workspace_size(n, spec.H, spec.d_v, spec.k)
+                 for n in {spec.T} | {c1 - c0 for c0, c1, _ in self.chunks})
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev) if ws else None
         self.prefill = spec.query_group > 1
         self.q_idx, self.w, self.q_mla = x["q_idx"], x["w"], x["q_mla"]
@@ -269,7 +282,33 @@ class Layer:
         fn = self.dsa.dsa_sparse_mla_prefill if self.prefill else self.dsa.dsa_sparse_mla_decode
         fn(q, lat, self.batch, idx, self.spec.scale, out, lse, self.ws, k=self.spec.k)
 
-    def step_sparse(self, ev=None):
+    def _mla_first(self, idx, mla_ready, out_host, d2h_stream):
+        """This layer's MLA (after its queries are in place); with out_host, its output goes back to
+        the host on d2h_stream chunk by chunk, each copy overlapping the next chunk's MLA and the
+        shared layers' MLAs; the compute stream waits for the copies at the end of the step."""
+        torch = self.torch
+        self._mla_inputs_ready(mla_ready)
+        if out_host is None:
+            self._mla(self.q_mla, self.lat, self.out, self.lse, idx)
+            return None
+        fn = self.dsa.dsa_sparse_mla_prefill if self.prefill else self.dsa.dsa_sparse_mla_decode
+        cur = torch.cuda.current_stream()
+        for (c0, c1, b), done in zip(self.chunks, self.chunk_done):
+            fn(self.q_mla[c0:c1], self.lat, b, None if idx is None else idx[c0:c1], self.spec.scale,
+               self.out[c0:c1], self.lse[c0:c1], self.ws, k=self.spec.k)
+            done.record(cur)
+            d2h_stream.wait_event(done)
+            with torch.cuda.stream(d2h_stream):
+                out_host[c0:c1].copy_(self.out[c0:c1], non_blocking=True)
+        self.back.record(d2h_stream)
+        return self.back
+
+    def _mla_inputs_ready(self, ready):
+        """The MLA reads queries that an end-to-end step copies on a side stream (None: resident)."""
+        if ready is not None:
+            self.torch.cuda.current_stream().wait_event(ready)
+
+    def step_sparse(self, ev=None, mla_ready=None, out_host=None, d2h_stream=None):
         """Indexer fused with the top-K selection (the indexer builds each query's order-key digit
         histogram, the selection places its threshold from it and clears it) -> sparse MLA (and
         the shared layers' sparse MLA on the same selection).  With events (per-kernel breakdown)
@@ -284,9 +323,11 @@ class Layer:
             ev[0].record()
             d.dsa_topk_select(self.scores, self.batch.q_pos, self.spec.k, self.idx, key_hist=self.khist)
             ev[1].record()
-        self._mla(self.q_mla, self.lat, self.out, self.lse, self.idx)
+        back = self._mla_first(self.idx, mla_ready, out_host, d2h_stream)
         for q, lat, out, lse in self.shared:
             self._mla(q, lat, out, lse, self.idx)
+        if back is not None:
+            self.torch.cuda.current_stream().wait_event(back)
 
     def step_unfused(self):
         """The same layer with the selection sampling its threshold (no histogram from the
@@ -298,13 +339,15 @@ class Layer:
         for q, lat, out, lse in self.shared:
             self._mla(q, lat, out, lse, self.idx)
 
-    def step(self, ev=None):
+    def step(self, ev=None, mla_ready=None, out_host=None, d2h_stream=None):
         if not self.dense:
-            return self.step_sparse(ev)
+            return self.step_sparse(ev, mla_ready, out_host, d2h_stream)
         if ev is not None:
             ev[0].record()
             ev[1].record()
-        self._mla(self.q_mla, self.lat, self.out, self.lse, None)
+        back = self._mla_first(None, mla_ready, out_host, d2h_stream)
+        if back is not None:
+            self.torch.cuda.current_stream().wait_event(back)
 
     def step_full_layer(self):
         """One full layer alone (indexer, top-K, sparse MLA): the IndexShare comparison."""
@@ -408,19 +451,38 @@ def run_cuda(args):
     ms_per_step = total_s * 1e3 / K
 
     # end to end through the public API: per-step query-side inputs from pinned host memory,
-    # the KV caches resident in HBM (state), output read back every step
-    names = ("q_req", "q_pos", "block_table", "q_mla") + (() if layer.dense else ("q_idx", "w"))
+    # the KV caches resident in HBM (state), output read back every step.  The indexer's inputs
+    # (and the batch description) are copied on the compute stream first; the MLA's queries,
+    # which nothing reads before the selection is done, follow on a second stream that the compute
+    # stream waits for just before the MLA, so that their copy overlaps the indexer and the
+    # selection; the output goes back on a third stream, chunk by chunk when the MLA runs in query
+    # chunks, or behind the shared layers' MLAs.  Small copies (under 1 MB of MLA queries; one
+    # chunk and no shared layers) stay on the compute stream: there the extra stream hand-offs
+    # would cost more than they hide.
+    first = ("q_req", "q_pos", "block_table") + (() if layer.dense else ("q_idx", "w"))
     if not layer.dense and x.get("q_idx_scale") is not None:
-        names += ("q_idx_scale",)
+        first += ("q_idx_scale",)
 
-    def query_inputs(c):  # device tensors of one copy that the host supplies every step
-        return [c[n] for n in names] + [sh["q_mla"] for sh in c.get("shared", [])]
-    host_in = [t.cpu().pin_memory() for t in query_inputs(x)]
-    dev_in = [query_inputs(c) for c in copies]
+    def first_inputs(c):  # device tensors of one copy that the host supplies every step
+        return [c[n] for n in first]
+
+    def mla_inputs(c):
+        return [c["q_mla"]] + [sh["q_mla"] for sh in c.get("shared", [])]
+    host_first = [t.cpu().pin_memory() for t in first_inputs(x)]
+    host_mla = [t.cpu().pin_memory() for t in mla_inputs(x)]
+    dev_first = [first_inputs(c) for c in copies]
+    dev_mla = [mla_inputs(c) for c in copies]
     host_out = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    mla_bytes = sum(t.numel() * t.element_size() for t in host_mla)
+    h2d = sum(t.numel() * t.element_size() for t in host_first) + mla_bytes
     d2h = host_out.numel() * host_out.element_size()
+    side_in = mla_bytes >= (1 << 20)
+    side_out = len(layer.chunks) > 1 or bool(layer.shared)
     e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    copy_stream = torch.cuda.Stream()
+    d2h_stream = torch.cuda.Stream()
+    first_done = [torch.cuda.Event() for _ in range(K)]
+    mla_ready = [torch.cuda.Event() for _ in range(K)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -428,10 +490,23 @@ def run_cuda(args):
         lay = layers[i % ncopy]
         torch.cuda.synchronize()  # end to end: every step starts from an idle device and host
         e2e_ev[i][0].record(stream)
-        for dst, src in zip(dev_in[i % ncopy], host_in):
+        for dst, src in zip(dev_first[i % ncopy], host_first):
             dst.copy_(src, non_blocking=True)
-        lay.step()
-        host_out.copy_(lay.out, non_blocking=True)
+        if side_in:
+            first_done[i].record(stream)
+            copy_stream.wait_event(first_done[i])  # after the indexer's inputs, inside the timed region
+            with torch.cuda.stream(copy_stream):
+                for dst, src in zip(dev_mla[i % ncopy], host_mla):
+                    dst.copy_(src, non_blocking=True)
+            mla_ready[i].record(copy_stream)
+        else:
+            for dst, src in zip(dev_mla[i % ncopy], host_mla):
+                dst.copy_(src, non_blocking=True)
+        if side_out:
+            lay.step(mla_ready=mla_ready[i] if side_in else None, out_host=host_out, d2h_stream=d2h_stream)
+        else:
+            lay.step(mla_ready=mla_ready[i] if side_in else None)
+            host_out.copy_(lay.out, non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     e2e_s = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / 1e3, world, dev)
@@ -524,7 +599,11 @@ def run_cuda(args):
             "planted_tail": planted,
             "e2e": {"value": e2e_value, "unit": "query-tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h,
-                    "note": "query-side inputs copied from pinned host memory every step; KV caches resident"},
+                    "note": ("query-side inputs copied from pinned host memory every step (MLA queries "
+                             "%s, output read back %s); KV caches resident" % (
+                                 "on a second stream, overlapping the indexer and the selection" if side_in
+                                 else "in order", "on a third stream, per MLA query chunk (%d), overlapping "
+                                 "the following work" % len(layer.chunks) if side_out else "at the end"))},
             "gpu_launches": launches,
             "roofline": roof,
             "breakdown": breakdown,
