@@ -88,6 +88,13 @@ def work_model(spec):
     mla_hbm_rows = sum(min(sel_req[r], per_req[r]) for r in sel_req)
     mla_bytes = mla_hbm_rows * spec.dqk * act + T * spec.H * (spec.dqk + spec.d_v) * act + T * spec.H * 4
     mla_flops = 2.0 * spec.H * mla_rows * (spec.dqk + spec.d_v)
+    # rows the tensor-core MLA gathers into shared memory: whole 64-row tiles of each query's
+    # selection slots (K of them; in the dense case its visible positions), by both value-half CTAs
+    tc_mla = spec.act_dtype == "bf16" and spec.H in (64, 128) and spec.d_v == 512 and spec.dqk == 576
+    dense = max(vis) <= spec.k
+    slots = [min(v, spec.k) for v in vis] if dense else [spec.k] * T
+    mla_gather_bytes = (2 * sum(-(-n // 64) * 64 for n in slots) * spec.dqk * act * spec.share_layers
+                        if tc_mla else 0)
     if max(vis) <= spec.k:
         # the dense case: every query keeps all its positions, no indexer or selection runs
         idx_bytes = idx_flops = topk_bytes = 0
@@ -96,7 +103,7 @@ def work_model(spec):
     mla_flops *= spec.share_layers
     return dict(indexer_bytes=idx_bytes, indexer_flops=idx_flops, topk_bytes=topk_bytes,
                 mla_bytes=mla_bytes, mla_flops=mla_flops, key_tokens=key_tokens, pairs=pairs,
-                mla_rows=mla_rows, mla_hbm_rows=mla_hbm_rows)
+                mla_rows=mla_rows, mla_hbm_rows=mla_hbm_rows, mla_gather_bytes=mla_gather_bytes)
 
 
 def resident_bytes(spec, x):
@@ -356,6 +363,29 @@ class Layer:
         self._mla(self.q_mla, self.lat, self.out, self.lse, self.idx)
 
 
+def gather_ceiling(dsa, lat, dev, tiles=32, seed=7):
+    """Rate of the sparse MLA's row gathers alone on every SM (dsa_selftest_gather_rate): random
+    rows of the latent pool, `tiles` 64-row tiles per CTA, one CTA per SM; GB/s over the launch
+    (CUDA events) and the mean bytes per SM cycle of the CTAs."""
+    import torch
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    pool_rows = lat.data.shape[0] * lat.data.shape[1]
+    g = torch.Generator(device=dev).manual_seed(seed)
+    rows = torch.randint(0, pool_rows, (sms * tiles * 64,), generator=g, device=dev, dtype=torch.int32)
+    cycles = torch.zeros(sms, dtype=torch.int64, device=dev)
+    dsa.dsa_selftest_gather_rate(lat, rows, tiles, sms, cycles)  # warm-up
+    b = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    b.record()
+    dsa.dsa_selftest_gather_rate(lat, rows, tiles, sms, cycles)
+    e.record()
+    torch.cuda.synchronize()
+    tile_bytes = 64 * 1152
+    gbs = sms * tiles * tile_bytes / (b.elapsed_time(e) / 1e3) / 1e9
+    c = cycles.double().cpu()
+    return {"gbs": gbs, "per_sm_cycle": float((tiles * tile_bytes / c[c > 0]).mean())}
+
+
 def _time_steps(fn, K, stream):
     """Device time of K back-to-back calls of fn, after a stream gate (CUDA events, ms)."""
     import torch
@@ -548,6 +578,16 @@ def run_cuda(args):
         breakdown[name + "_us"] = r["us"]
         breakdown[name + "_frac"] = r["frac"]
         breakdown[name + "_bound"] = r["bound"]
+    # The sparse MLA is bound by the rate at which the SMs gather its rows (TMA tile::gather4 of
+    # 128-byte boxes), not by HBM or the tensor cores: its gathered bytes per second against that
+    # rate, measured in this run by the library's gather diagnostic (the MLA's gathers alone) on
+    # random rows of this workload's latent pool, over every SM.
+    if model["mla_gather_bytes"] and mla_ms:
+        ceil = gather_ceiling(dsa, layer.lat, dev)
+        achieved = model["mla_gather_bytes"] / (statistics.mean(mla_ms) / 1e3) / 1e9
+        breakdown["mla_gather"] = {"bytes": model["mla_gather_bytes"], "achieved_gbs": achieved,
+                                   "ceiling_gbs": ceil["gbs"], "ceiling_bytes_per_sm_cycle": ceil["per_sm_cycle"],
+                                   "frac": achieved / ceil["gbs"]}
 
     # comparisons on the same inputs: the sparse path where the dense case applies, and one full
     # layer alone where a group of layers shares one selection

@@ -235,6 +235,19 @@ size_t dsa_mla_workspace_size(int32_t num_queries, int32_t H, int32_t d_v, int32
  * usable.  Read the word with dsa_get_device_error. */
 dsa_status dsa_selftest_bounded_wait(int64_t limit_cycles, dsa_stream stream);
 
+/* Diagnostic of the sparse MLA's row-gather rate (no counterpart on the pages): enqueues one
+ * kernel of num_ctas CTAs (1 .. 1024) that gathers latent rows exactly as the tensor-core sparse
+ * MLA does -- 64-row tiles, each row's nine 128-byte column blocks by TMA tile::gather4, a
+ * two-stage shared-memory ring -- and does nothing else with them.  CTA c gathers the pool rows
+ * rows[(c * tiles_per_cta + j) * 64 + i] (tile j = 0 .. tiles_per_cta-1, i = 0 .. 63; a device
+ * int32 array of num_ctas * tiles_per_cta * 64 entries, each a row index of the pool, block *
+ * 64 + offset) and writes its SM cycles from the start of its gathers to the landing of its last
+ * tile to cycles[c] (device int64; -1 when a bounded wait gave up).  A row index outside the pool
+ * sets DSA_DEVERR_INDEX and reads as zeros.  latent: bf16, block_size 64, dim 576, data 16-byte
+ * aligned (the tensor-core MLA's shape).  tiles_per_cta: 1 .. 65536. */
+dsa_status dsa_selftest_gather_rate(const dsa_paged_cache* latent, const int32_t* rows, int32_t tiles_per_cta,
+                                    int32_t num_ctas, int64_t* cycles, dsa_stream stream);
+
 /* Synchronises `stream`, then reads the device error word of the current device into *code
  * (0 = no fault).  Not for use inside stream capture. */
 dsa_status dsa_get_device_error(int32_t* code, dsa_stream stream);

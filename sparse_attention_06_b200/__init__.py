@@ -35,7 +35,7 @@ EXPORTED = (
     "dsa_sparse_mla_prefill", "dsa_mla_workspace_size", "dsa_get_device_error",
     "dsa_clear_device_error", "dsa_status_string", "dsa_last_error_message", "dsa_abi_version",
     "dsa_kernel_launch_count", "dsa_sparse_mla_decode_noalloc", "dsa_selftest_bounded_wait",
-    "dsa_indexer_topk_workspace_size",
+    "dsa_indexer_topk_workspace_size", "dsa_selftest_gather_rate",
 )
 
 
@@ -87,6 +87,7 @@ def load_library():
         "dsa_get_device_error": [ctypes.POINTER(I32), P],
         "dsa_clear_device_error": [P],
         "dsa_selftest_bounded_wait": [I64, P],
+        "dsa_selftest_gather_rate": [PC, P, I32, I32, P, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -277,6 +278,20 @@ def dsa_selftest_bounded_wait(limit_cycles, stream=None):
     """Diagnostic: a kernel whose bounded wait on a phase that never completes gives up after
     ``limit_cycles`` SM cycles and sets DEVERR_TIMEOUT (include/dsa.h)."""
     _check(load_library().dsa_selftest_bounded_wait(int(limit_cycles), _stream(stream)))
+
+
+def dsa_selftest_gather_rate(latent: PagedCache, rows, tiles_per_cta, num_ctas, cycles, stream=None):
+    """Diagnostic: gathers latent pool rows with the sparse MLA's TMA pattern and nothing else;
+    rows: int32 [num_ctas * tiles_per_cta * 64] pool row indices; cycles: int64 [num_ctas]
+    receives each CTA's SM cycles (include/dsa.h)."""
+    if rows.dtype != torch.int32 or rows.numel() < num_ctas * tiles_per_cta * 64:
+        raise ValueError("rows must be int32 with num_ctas * tiles_per_cta * 64 entries")
+    if cycles.dtype != torch.int64 or cycles.numel() < num_ctas:
+        raise ValueError("cycles must be int64 with num_ctas entries")
+    lc = latent._c()
+    _check(load_library().dsa_selftest_gather_rate(ctypes.byref(lc), _dev_ptr(rows, "rows"), int(tiles_per_cta),
+                                                   int(num_ctas), _dev_ptr(cycles, "cycles"), _stream(stream)))
+    return cycles
 
 
 def dsa_clear_device_error(stream=None):

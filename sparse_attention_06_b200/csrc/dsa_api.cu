@@ -386,6 +386,24 @@ dsa_status dsa_selftest_bounded_wait(int64_t limit_cycles, dsa_stream stream) {
                      "dsa_selftest_bounded_wait launch", 1);
 }
 
+dsa_status dsa_selftest_gather_rate(const dsa_paged_cache* latent, const int32_t* rows, int32_t tiles_per_cta,
+                                    int32_t num_ctas, int64_t* cycles, dsa_stream stream) {
+  if (!latent || !latent->data || !rows || !cycles) return fail(DSA_ERR_INVALID_ARG, "gather rate: NULL argument%s");
+  if (latent->dtype != DSA_BF16 || latent->block_size != 64 || latent->dim != 576 || latent->num_blocks < 1 ||
+      (reinterpret_cast<uintptr_t>(latent->data) & 15u))
+    return fail(DSA_ERR_INVALID_ARG, "gather rate: latent must be bf16, 64-token blocks of 576, 16-byte aligned%s");
+  if ((uint64_t)latent->num_blocks * 64u >= 0x7FFFFFFFull)
+    return fail(DSA_ERR_INVALID_ARG, "gather rate: pool rows must fit 31 bits%s");
+  if (tiles_per_cta < 1 || tiles_per_cta > 65536 || num_ctas < 1 || num_ctas > 1024)
+    return fail(DSA_ERR_INVALID_ARG, "gather rate: tiles_per_cta in [1, 65536], num_ctas in [1, 1024]%s");
+  int* err;
+  int sms;
+  if (!device_state(&err, &sms)) return fail(DSA_ERR_CUDA, "no CUDA device%s");
+  return cuda_status(launch_gather_rate_selftest(*latent, rows, tiles_per_cta, num_ctas, cycles, err,
+                                                 static_cast<cudaStream_t>(stream)),
+                     "dsa_selftest_gather_rate launch", 1);
+}
+
 size_t dsa_mla_workspace_size(int32_t num_queries, int32_t H, int32_t d_v, int32_t k) {
   if (num_queries <= 0 || (H != 128 && H != 64) || d_v != 512 || k < 1) return 0;
   int dev = 0, sms = 148;

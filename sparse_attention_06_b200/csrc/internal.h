@@ -103,6 +103,8 @@ MlaPlan mla_plan(bool decode, const void* q, int32_t q_dtype, int32_t H, int32_t
 
 // diagnostic: one thread waits on an mbarrier that nothing arrives on, bounded by limit_cycles
 cudaError_t launch_bounded_wait_selftest(long long limit_cycles, int* err, cudaStream_t s);
+cudaError_t launch_gather_rate_selftest(const dsa_paged_cache& latent, const int32_t* rows, int tiles, int ctas,
+                                        int64_t* cycles, int* err, cudaStream_t s);
 
 // tensor-map encoding through the driver entry point (no link-time libcuda dependency)
 bool encode_tmap_2d(void* tmap_out, const void* base, int elem_bytes, uint64_t inner,

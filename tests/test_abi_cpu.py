@@ -74,6 +74,13 @@ def test_invalid_arguments_rejected_on_host(lib):
     st = lib.dsa_sparse_mla_decode(fake, 1, 128, 512, 64, ctypes.byref(lc), ctypes.byref(b), fake, 2048,
                                    ctypes.c_float(-1.0), fake, None, None, 0, None)
     assert st == dsa.DSA_ERR_INVALID_ARG
+    # the gather-rate diagnostic checks its shape and sizes on the host
+    gc = dsa._PagedCache(16, None, 4, 64, 576, dsa.DSA_BF16, 0)
+    assert lib.dsa_selftest_gather_rate(ctypes.byref(gc), None, 1, 1, fake, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_selftest_gather_rate(ctypes.byref(gc), fake, 0, 1, fake, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_selftest_gather_rate(ctypes.byref(gc), fake, 1, 2000, fake, None) == dsa.DSA_ERR_INVALID_ARG
+    gc = dsa._PagedCache(16, None, 4, 64, 512, dsa.DSA_BF16, 0)
+    assert lib.dsa_selftest_gather_rate(ctypes.byref(gc), fake, 1, 1, fake, None) == dsa.DSA_ERR_INVALID_ARG
     # max_blocks * block_size must cover max_context
     b = dsa._Batch(1, 1, 16, 16, 16, 2, 256, 1, 0)
     st = lib.dsa_sparse_mla_decode(fake, 1, 128, 512, 64, ctypes.byref(lc), ctypes.byref(b), fake, 2048,

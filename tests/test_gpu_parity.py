@@ -317,6 +317,33 @@ def test_bounded_wait_runs_out_and_context_stays_usable():
     parity_case(x, kind="bf16")
 
 
+def test_gather_rate_diagnostic():
+    # the sparse MLA's row gathers alone: every CTA reports its cycles, the implied rate is a
+    # plausible number of bytes per SM cycle, and a row index outside the pool is flagged
+    # (and read as zeros) without stopping the kernel
+    g = torch.Generator().manual_seed(61)
+    nblk, ctas, tiles = 40, 4, 8
+    pool = torch.randn(nblk, 64, 576, generator=g).to(torch.bfloat16).cuda()
+    lat = dsa.PagedCache(pool)
+    rows = torch.randint(0, nblk * 64, (ctas * tiles * 64,), generator=g, dtype=torch.int32).cuda()
+    cycles = torch.zeros(ctas, dtype=torch.int64, device="cuda")
+    dsa.dsa_clear_device_error()
+    dsa.dsa_selftest_gather_rate(lat, rows, tiles, ctas, cycles)
+    assert dsa.dsa_get_device_error() == 0
+    c = cycles.cpu()
+    assert (c > 0).all()
+    rate = tiles * 64 * 1152 / c.double()  # bytes per SM cycle of each CTA
+    assert ((rate > 1.0) & (rate < 256.0)).all(), rate
+    rows[5] = -1
+    rows[77] = nblk * 64
+    dsa.dsa_selftest_gather_rate(lat, rows, tiles, ctas, cycles)
+    assert dsa.dsa_get_device_error() == dsa.DEVERR_INDEX
+    assert (cycles.cpu() > 0).all()
+    dsa.dsa_clear_device_error()
+    with pytest.raises(dsa.DsaError):
+        dsa.dsa_selftest_gather_rate(lat, rows, 0, ctas, cycles)
+
+
 # ---------------------------------------------------------------------------------------------
 # the dense case and IndexShare
 # ---------------------------------------------------------------------------------------------
