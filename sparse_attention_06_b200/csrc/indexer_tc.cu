@@ -89,7 +89,7 @@ struct Cfg {
   // Epilogue sets of four warps (each set covers the 128 TMEM lanes).  With one query per tile
   // the sets take tiles in turn (three for e4m3 keys and queries, whose 16 KB tiles come twice as
   // fast as bf16 ones); with four queries two sets take every tile, each scoring two queries.
-  static constexpr int EPI_SETS = FP8 && NQ == 1 && !SPLIT1 ? 3 : 2;
+  static constexpr int EPI_SETS = NQ == 1 ? (FP8 && !SPLIT1 ? 3 : 2) : 2;
   static constexpr int EPI_WARPS = 4 * EPI_SETS;
   static constexpr bool EPI_ALT = NQ == 1;
   static constexpr int TSTEP = EPI_ALT ? EPI_SETS : 1;        // tiles between one set's tiles
@@ -110,8 +110,9 @@ struct Cfg {
   static constexpr int Q_CHUNK = N * 128;                     // one 128-byte-row block of a query tile
   static constexpr int Q_BYTES = FP8 ? TERMS * Q_CHUNK : 2 * Q_CHUNK;
   static constexpr int TMEM_COLS = NACC * NMMA <= 256 ? (NACC * NMMA <= 128 ? 128 : 256) : 512;
-  static constexpr int EPI_NQ = EPI_ALT ? NQ : NQ / 2;       // queries per epilogue warp
-  static constexpr int EPI_ARRIVE = EPI_ALT ? 4 : 8;          // epilogue arrivals per tile
+  static constexpr int EPI_NQ = EPI_ALT ? NQ : NQ / EPI_SETS;  // queries per epilogue warp
+  static_assert(EPI_ALT || EPI_NQ * EPI_SETS == NQ, "the epilogue sets score every query of a group once");
+  static constexpr int EPI_ARRIVE = EPI_ALT ? 4 : EPI_WARPS;  // epilogue arrivals per tile
   // (one prep warp with one query per tile keeps the CTA at 16 warps, four per SM sub-partition,
   // which leaves every thread 128 registers)
   static constexpr int PREP_WARPS = FP8 ? (NQ == 1 ? 1 : 4) : 0;
@@ -727,6 +728,21 @@ __global__ void __launch_bounds__(Cfg<NQ, KM>::THREADS, 1)
         // head pairs in packed f32x2 FMAs, four independent pair accumulators; the heads in two
         // halves of 32 columns (with SPLIT_N, each the sum of its two term columns)
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        if constexpr (!C::SPLIT_N && NQ > 1) {
+          // (four queries per tile: all 64 head columns in flight before one wait)
+          uint32_t v[64];
+#pragma unroll
+          for (int c16 = 0; c16 < 4; ++c16)
+            tmem_ld16(tbase + qi * 64 + c16 * 16, *reinterpret_cast<uint32_t(*)[16]>(&v[c16 * 16]));
+          tmem_wait_ld();
+#pragma unroll
+          for (int h4 = 0; h4 < 16; ++h4) {
+            const float4 wv = w4[h4];
+            uint64_t* ac = acc + (h4 & 1) * 2;
+            ac[0] = ffma2(wv.x, wv.y, fmaxf(__uint_as_float(v[4 * h4 + 0]), 0.0f), fmaxf(__uint_as_float(v[4 * h4 + 1]), 0.0f), ac[0]);
+            ac[1] = ffma2(wv.z, wv.w, fmaxf(__uint_as_float(v[4 * h4 + 2]), 0.0f), fmaxf(__uint_as_float(v[4 * h4 + 3]), 0.0f), ac[1]);
+          }
+        } else
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           uint32_t v[32];
