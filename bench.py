@@ -261,11 +261,9 @@ class Layer:
         # back to the host while the next is computed: as many chunks (1, 2 or 4, whole query
         # groups) as keep every chunk at four or more (query, value half) units per SM
         sms = torch.cuda.get_device_properties(dev).multi_processor_count if dev.type == "cuda" else 148
-        nch = next(c for c in (4, 2, 1) if c == 1 or 2 * spec.T // c >= 4 * sms)
-        g = max(1, spec.query_group)
-        cuts = sorted({min(spec.T, (spec.T * i // nch) // g * g) for i in range(nch + 1)})
         self.chunks = [(c0, c1, dsa.Batch(x["q_req"][c0:c1], x["q_pos"][c0:c1], x["block_table"], self.max_ctx,
-                                          spec.query_group)) for c0, c1 in zip(cuts[:-1], cuts[1:]) if c1 > c0]
+                                          spec.query_group))
+                       for c0, c1 in mla_query_chunks(spec.T, spec.query_group, sms)]
         self.chunk_done = [torch.cuda.Event() for _ in self.chunks] if dev.type == "cuda" else []
         self.back = torch.cuda.Event() if dev.type == "cuda" else None
         ws = max(dsa.dsa_mla_workspace_size(n, spec.H, spec.d_v, spec.k)
@@ -361,6 +359,16 @@ class Layer:
         self.dsa.dsa_indexer_topk(self.q_idx, self.w, self.keys, self.batch, self.spec.k, self.scores, self.idx,
                                   q_scale=self.q_scale, workspace=self.khist)
         self._mla(self.q_mla, self.lat, self.out, self.lse, self.idx)
+
+
+def mla_query_chunks(T, query_group, sms):
+    """Query ranges [c0, c1) of an end-to-end step's MLA calls: 1, 2 or 4 chunks of whole query
+    groups, as many as keep every chunk at four or more (query, value half) units per SM, so that
+    each chunk still fills the GPU while the previous chunk's output goes back to the host."""
+    nch = next(c for c in (4, 2, 1) if c == 1 or 2 * T // c >= 4 * sms)
+    g = max(1, query_group)
+    cuts = sorted({min(T, (T * i // nch) // g * g) for i in range(nch + 1)} | {T})
+    return [(c0, c1) for c0, c1 in zip(cuts[:-1], cuts[1:]) if c1 > c0]
 
 
 def gather_ceiling(dsa, lat, dev, tiles=32, seed=7):

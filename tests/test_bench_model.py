@@ -55,3 +55,18 @@ def test_work_model_dense_and_indexshare():
     grp = bench.work_model(di.indexshare())
     assert grp["indexer_bytes"] == one["indexer_bytes"]                  # one indexer per group
     assert grp["mla_flops"] == 4 * one["mla_flops"] and grp["mla_bytes"] == 4 * one["mla_bytes"]
+
+
+def test_mla_query_chunks_cover_the_batch_in_whole_groups():
+    # the end-to-end step's MLA chunks: contiguous, covering every query once, whole query groups,
+    # and only as many as keep each chunk at four or more units per SM
+    for T, g, sms in ((4096, 4, 148), (64, 1, 148), (16, 1, 148), (1, 1, 148), (1200, 4, 148), (2000, 4, 148),
+                      (1184, 1, 148), (4100, 4, 148)):
+        ch = bench.mla_query_chunks(T, g, sms)
+        assert ch[0][0] == 0 and ch[-1][1] == T
+        assert all(a[1] == b[0] for a, b in zip(ch[:-1], ch[1:]))
+        assert all(c0 % g == 0 for c0, _ in ch)
+        if len(ch) > 1:
+            assert all(2 * (c1 - c0) >= 4 * sms - 2 * g for c0, c1 in ch)
+    assert len(bench.mla_query_chunks(4096, 4, 148)) == 4
+    assert len(bench.mla_query_chunks(64, 1, 148)) == 1
