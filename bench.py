@@ -394,11 +394,14 @@ def gather_ceiling(dsa, lat, dev, tiles=32, seed=7):
     return {"gbs": gbs, "per_sm_cycle": float((tiles * tile_bytes / c[c > 0]).mean())}
 
 
-def _time_steps(fn, K, stream):
-    """Device time of K back-to-back calls of fn, after a stream gate (CUDA events, ms)."""
+def _time_steps(fn, K, stream, warmup=3):
+    """Device time of K back-to-back calls of fn, after `warmup` untimed calls (so that a kernel
+    no earlier pass ran is loaded and warm) and a stream gate (CUDA events, ms)."""
     import torch
     b = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
+    for i in range(warmup):
+        fn(i)
     torch.cuda.synchronize()
     torch.cuda._sleep(GATE_CYCLES)
     b.record(stream)

@@ -258,10 +258,10 @@ __device__ __forceinline__ void store_o(const Params& p, uint32_t lane_base, int
   }
 }
 
-template <int H, bool kStagedQ>
+template <int H, bool kStagedQ, bool kDense>
 __global__ void __launch_bounds__(kThreads, 1)
     mla_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap lmap,
-                  const Params p) {
+                  const __grid_constant__ CUtensorMap pmap, const Params p) {
   using HC = HCfg<H>;
   constexpr int RQ = HC::RQ;
   constexpr int Q_CHUNK = HC::Q_CHUNK;
@@ -410,10 +410,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         ps_j = ps_j1;
         ps_j1 = ps_j2;
         blk_j = blk_j1;
-        // this warp's 16 rows: four gather4 groups of four rows x nine 64-dim column blocks
+        // Without a selection a tile is 64 consecutive positions starting at a multiple of 64:
+        // one whole page when every position is visible and the page exists.  Such a tile comes
+        // in as nine 64-row boxes (warp 0), every other tile as gathered rows, this warp's 16 as
+        // four gather4 groups of four rows x nine 64-dim column blocks (rows past the pool,
+        // never read, for the unused slots).  The byte count is the same either way.
         const int32_t rc = row >= 0 ? (int32_t)row : p.oob_row;
         uint8_t* stage = k_ring + s * K_BYTES + gw * kKeysPerWarp * 128;
+        bool whole_page = false;
+        if constexpr (kDense)
+          whole_page = sp * p.ks + j * kTile + kTile - 1 <= pos && __all_sync(0xFFFFFFFFu, !mine || row >= 0);
         if (lane == 0) mbar_arrive_expect_tx(&k_full[s], kKeysPerWarp * kDqk * 2);
+        if (whole_page) {
+          const int32_t prow = __shfl_sync(0xFFFFFFFFu, rc, 0) & ~(kPage - 1);  // the page's first row
+          if (gw == 0 && lane == 0) {
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) tma_load_2d(k_ring + s * K_BYTES + c * K_CHUNK, &pmap, &k_full[s], c * 64, prow);
+          }
+        } else
 #pragma unroll
         for (int g4 = 0; g4 < kKeysPerWarp / 4; ++g4) {
           const int32_t r0 = __shfl_sync(0xFFFFFFFFu, rc, 4 * g4 + 0);
@@ -817,11 +831,14 @@ template <int H>
 cudaError_t launch_mla_tc_h(const MlaArgs& a, int nsplit, int num_sms, cudaStream_t s) {
   using HC = HCfg<H>;
   const int T = a.batch.num_queries;
-  alignas(64) CUtensorMap qmap, lmap;
+  alignas(64) CUtensorMap qmap, lmap, pmap;
   if (!encode_tmap_2d(&qmap, a.q, 2, kDqk, (uint64_t)T * H, kDqk * 2, 64, H, true)) return cudaErrorInvalidValue;
   const uint64_t pool_rows = (uint64_t)a.latent.num_blocks * kPage;
   if (pool_rows >= 0x7FFFFFFFull) return cudaErrorInvalidValue;  // row coordinates are 32-bit
   if (!encode_tmap_2d(&lmap, a.latent.data, 2, kDqk, pool_rows, (uint64_t)kDqk * 2, 64, 1, true))
+    return cudaErrorInvalidValue;
+  // whole 64-token pages (the dense case): 64-row boxes of one 64-dim column block
+  if (!encode_tmap_2d(&pmap, a.latent.data, 2, kDqk, pool_rows, (uint64_t)kDqk * 2, 64, kPage, true))
     return cudaErrorInvalidValue;
   Params p;
   p.latent = static_cast<const __nv_bfloat16*>(a.latent.data);
@@ -853,12 +870,14 @@ cudaError_t launch_mla_tc_h(const MlaArgs& a, int nsplit, int num_sms, cudaStrea
   }
   const int units = T * nsplit * 2;
   const int grid = units < num_sms ? units : num_sms;
-  auto kernel = units <= grid ? mla_tc_kernel<H, true> : mla_tc_kernel<H, false>;  // one unit per CTA: staged Q
+  // one unit per CTA: staged Q; without a selection: whole pages by 64-row boxes
+  auto kernel = units <= grid ? (p.dense ? mla_tc_kernel<H, true, true> : mla_tc_kernel<H, true, false>)
+                              : (p.dense ? mla_tc_kernel<H, false, true> : mla_tc_kernel<H, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HC::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attrs[2];
   const cudaLaunchConfig_t cfg = launch_config(dim3(grid), dim3(kThreads), HC::SMEM, s, attrs);
-  e = cudaLaunchKernelEx(&cfg, kernel, qmap, lmap, p);
+  e = cudaLaunchKernelEx(&cfg, kernel, qmap, lmap, pmap, p);
   if (e != cudaSuccess || nsplit == 1) return e;
   cudaLaunchAttribute cattrs[2];
   const cudaLaunchConfig_t ccfg = launch_config(dim3(T, H), dim3(kCombThreads), 0, s, cattrs);
