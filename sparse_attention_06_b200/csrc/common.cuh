@@ -158,6 +158,24 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, ui
       : "memory");
 }
 
+// L2 cache policy that makes the lines a load brings in the first to be evicted: for data read once
+// (keys streamed past a single query), so that they do not push out what the next kernel reads.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// tma_load_2d with an L2 cache-policy hint (a policy from createpolicy).
+__device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const void* tmap, uint64_t* bar,
+                                                 int32_t c0, int32_t c1, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "l"(policy)
+      : "memory");
+}
+
 // TMA gather of four rows (tile::gather4; 2-D tensor map whose box is one row high): columns
 // [c0, c0 + box) of rows r0..r3 land as four consecutive box rows at smem_dst, completion counted
 // on `bar` in bytes.  Rows outside the tensor read as zeros.  No multicast.

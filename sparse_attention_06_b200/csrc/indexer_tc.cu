@@ -168,6 +168,7 @@ struct Params {
   int64_t num_blocks;
   int num_queries, num_reqs, max_blocks, max_context;
   int* err;
+  int stream_keys;               // each key page is read by one query tile: load keys evict-first
 };
 
 // One query group (NQ consecutive queries of one request) and its tile count.
@@ -461,6 +462,14 @@ __global__ void __launch_bounds__(Cfg<NQ, KM>::THREADS, 1)
       fetch();
       int last = -1, m = -1;  // (lane 0) group of the last query tile issued, query tiles issued
       int64_t i = 0;          // tiles whose copies were issued (the first tile of the batch below)
+      // keys read once (decode) are loaded evict-first, so that they do not push the scores this
+      // kernel writes out of L2 before the selection reads them
+      const bool hint = p.stream_keys != 0;
+      const uint64_t key_policy = hint ? l2_policy_evict_first() : 0ull;
+      auto load_key = [&](uint8_t* dst, int32_t c0, int32_t row, uint64_t* bar) {
+        if (hint) tma_load_2d_hint(dst, &kmap, bar, c0, row, key_policy);
+        else tma_load_2d(dst, &kmap, bar, c0, row);
+      };
       bool ok = true;
       while (ok && n_cnt > 0) {
         const int cnt = n_cnt;
@@ -512,17 +521,17 @@ __global__ void __launch_bounds__(Cfg<NQ, KM>::THREADS, 1)
               uint8_t* dst = op_ring + st * C::OP_BYTES;
               if constexpr (FP8) {
                 // a 64-token e4m3 page is one 8 KB box of 128-byte rows
-                if (t0 >= 0) tma_load_2d(dst, &kmap, &op_full[st], 0, t0 * kPage);
-                if (t1 >= 0) tma_load_2d(dst + 8192, &kmap, &op_full[st], 0, t1 * kPage);
+                if (t0 >= 0) load_key(dst, 0, t0 * kPage, &op_full[st]);
+                if (t1 >= 0) load_key(dst + 8192, 0, t1 * kPage, &op_full[st]);
               } else {
                 // a bf16 page is two 8 KB boxes (dims 0..63 and 64..127), one per column block
                 if (t0 >= 0) {
-                  tma_load_2d(dst, &kmap, &op_full[st], 0, t0 * kPage);
-                  tma_load_2d(dst + C::CHUNK_BYTES, &kmap, &op_full[st], 64, t0 * kPage);
+                  load_key(dst, 0, t0 * kPage, &op_full[st]);
+                  load_key(dst + C::CHUNK_BYTES, 64, t0 * kPage, &op_full[st]);
                 }
                 if (t1 >= 0) {
-                  tma_load_2d(dst + 8192, &kmap, &op_full[st], 0, t1 * kPage);
-                  tma_load_2d(dst + C::CHUNK_BYTES + 8192, &kmap, &op_full[st], 64, t1 * kPage);
+                  load_key(dst + 8192, 0, t1 * kPage, &op_full[st]);
+                  load_key(dst + C::CHUNK_BYTES + 8192, 64, t1 * kPage, &op_full[st]);
                 }
               }
               ++issued;
@@ -872,7 +881,9 @@ cudaError_t launch_impl(const IndexerArgs& a, int num_sms, cudaStream_t s) {
   if (!ok) return cudaErrorInvalidValue;
   Params p{a.batch.q_req, a.batch.q_pos, a.batch.block_table, a.q, a.q_scale, a.w, a.keys.scale, a.scores, a.ld,
            a.key_hist, a.keys.num_blocks, a.batch.num_queries, a.batch.num_reqs, a.batch.max_blocks,
-           a.batch.max_context, a.err};
+           a.batch.max_context, a.err,
+           // one query per request (decode): every key page is read by one query tile only
+           (NQ == 1 && a.batch.num_queries <= a.batch.num_reqs) ? 1 : 0};
   auto kern = indexer_tc_kernel<NQ, KM>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
