@@ -30,7 +30,8 @@
 //               the following batch already in flight), checks them and publishes 8-32 tiles'
 //               block ids in a tile-info ring in one lane-parallel pass, then (lane 0) issues the
 //               TMA copies of key pages (and, for bf16 keys, of query tiles) into 128B-swizzled
-//               shared memory
+//               shared memory; key pages that only one tile reads (one query per request) are
+//               copied with an L2 evict-first policy
 //   warp 1      TMEM allocation and the thread that issues tcgen05.mma / tcgen05.commit (with one
 //               query per tile, of the even tiles; the last warp issues the odd ones)
 //   epilogue    sets of 4 warps: with one query per tile three sets (e4m3 keys) or two (bf16)
