@@ -70,3 +70,23 @@ def test_mla_query_chunks_cover_the_batch_in_whole_groups():
             assert all(2 * (c1 - c0) >= 4 * sms - 2 * g for c0, c1 in ch)
     assert len(bench.mla_query_chunks(4096, 4, 148)) == 4
     assert len(bench.mla_query_chunks(64, 1, 148)) == 1
+
+
+def test_traffic_figures_follow_the_kernel_code(tmp_path, monkeypatch):
+    # a committed DRAM-traffic figure stays valid across edits of comments and white space, and
+    # is dropped (None) as soon as the kernel's code changes
+    import json
+    src = tmp_path / "k.cu"
+    src.write_text("// header\n__global__ void k(int* a) { a[0] = 1; }  /* note */\n")
+    d0 = bench.source_digest(str(src))
+    src.write_text("// another header\n__global__ void k(int* a)\n{\n  a[0] = 1;   // same code\n}\n")
+    assert bench.source_digest(str(src)) == d0
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"indexer@w": {"source": "k.cu", "source_digest": d0, "bytes_per_launch": 1234}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.ncu_traffic("indexer", "w") == 1234.0
+    assert bench.ncu_traffic("indexer", "other") is None
+    src.write_text("__global__ void k(int* a) { a[0] = 2; }\n")
+    assert bench.source_digest(str(src)) != d0
+    assert bench.ncu_traffic("indexer", "w") is None
